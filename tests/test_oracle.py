@@ -1,0 +1,301 @@
+"""Pins for the CPU oracle: each test checks it against something other than itself.
+
+Sources: "KVarN: Variance-Normalized KV-Cache Quantization Mitigates Error
+Accumulation in Reasoning Tasks" -- abstract (Hadamard rotation, dual-scaling
+variance normalisation over both axes, 2-bit) and the rndamp.com article,
+"How It Works" items 1-2, "Numbers" (second scale fused into dequantisation).
+The pages print no worked example, so the pins are closed forms, invariants,
+library routines and brute force (see tests/golden/README.md).
+"""
+import math
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle
+from bit_kv_cache_token_b200 import synth
+
+
+# ------------------------------------------------------------------ rotation
+@pytest.mark.parametrize("n", [2, 4, 32, 64, 128])
+def test_hadamard_is_sylvester_and_orthogonal(n):
+    H = oracle.hadamard_matrix(n)
+    np.testing.assert_array_equal(H, scipy.linalg.hadamard(n).astype(np.float64))
+    np.testing.assert_array_equal(H @ H.T, n * np.eye(n))
+
+
+@pytest.mark.parametrize("D,hb", [(64, 64), (128, 128), (96, 32), (128, 32), (128, 64)])
+def test_rotation_matches_library_blockdiag(D, hb):
+    rng = np.random.default_rng(D + hb)
+    x = rng.standard_normal((5, D))
+    H = scipy.linalg.hadamard(hb) / math.sqrt(hb)
+    M = scipy.linalg.block_diag(*([H] * (D // hb)))
+    np.testing.assert_allclose(oracle.rotate(x, hb), x @ M.T, rtol=0, atol=1e-12)
+    # orthogonal and self-inverse
+    np.testing.assert_allclose(np.linalg.norm(oracle.rotate(x, hb), axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)
+    np.testing.assert_allclose(oracle.rotate(oracle.rotate(x, hb), hb), x, atol=1e-12)
+
+
+def test_rotation_off_is_identity():
+    x = np.random.default_rng(1).standard_normal((3, 64))
+    np.testing.assert_array_equal(oracle.rotate(x, 0), x)
+
+
+@pytest.mark.parametrize("D,hb", [(64, 64), (128, 128), (96, 32)])
+def test_joint_rotation_preserves_dot_products(D, hb):
+    rng = np.random.default_rng(7)
+    q = rng.standard_normal((4, D))
+    k = rng.standard_normal((9, D)) * np.exp(rng.standard_normal(D))
+    np.testing.assert_allclose(oracle.rotate(q, hb) @ oracle.rotate(k, hb).T, q @ k.T, rtol=0, atol=1e-12 * D)
+
+
+# ------------------------------------------------------------ normalisation
+def _config0_k(seed=0):
+    k, v = synth.layer_kv(seed, 0, 1, 1, 256, 64, n_outliers=2, dtype=torch.float32)
+    return k[0, 0].double().numpy(), v[0, 0].double().numpy()
+
+
+@pytest.mark.parametrize("which", ["k", "v"])
+def test_variance_uniform_after_four_sweeps(which):
+    """Rows and columns of Y = Xrot / (r c) end within 1e-3 of uniform variance."""
+    kk, vv = _config0_k(0)
+    X = kk if which == "k" else vv
+    for b in range(2):
+        Xb = oracle.rotate(X[b * 128:(b + 1) * 128], 64)
+        r, c = oracle.normalize(Xb, 4)
+        Y = Xb / (r[:, None] * c[None, :])
+        col = Y.var(axis=0)
+        row = Y.var(axis=1)
+        np.testing.assert_allclose(col, 1.0, rtol=0, atol=1e-12)  # the last step is a column step
+        assert np.max(np.abs(row / row.mean() - 1.0)) <= 1e-3
+        # one sweep leaves the rows visibly less uniform than four (the iteration is doing work)
+        r1, c1 = oracle.normalize(Xb, 1)
+        row1 = (Xb / (r1[:, None] * c1[None, :])).var(axis=1)
+        assert np.max(np.abs(row1 / row1.mean() - 1.0)) > np.max(np.abs(row / row.mean() - 1.0))
+
+
+def _paired_rank_one(T=16, D=64, seed=3):
+    rng = np.random.default_rng(seed)
+    a = np.repeat(np.exp(rng.standard_normal(T // 2)), 2)
+    b = np.repeat(np.exp(rng.standard_normal(D // 2)), 2)
+    sign = (-1.0) ** np.add.outer(np.arange(T), np.arange(D))
+    return a, b, np.outer(a, b) * sign
+
+
+@pytest.mark.parametrize("sweeps", [1, 2, 4])
+def test_closed_form_paired_rank_one(sweeps):
+    """X_td = a_t b_d (-1)^(t+d), a and b positive and paired, rotation off:
+    r_t = a_t RMS(b), c_d = b_d / RMS(b) after the first sweep and at every later one,
+    Y = +-1 and the codes are 0 / 3 by the sign pattern."""
+    a, b, X = _paired_rank_one()
+    rms = math.sqrt(np.mean(b * b))
+    r, c = oracle.normalize(X, sweeps)
+    np.testing.assert_allclose(r, a * rms, rtol=1e-13)
+    np.testing.assert_allclose(c, b / rms, rtol=1e-13)
+    q = oracle.quantize_block(X, hb=0, sweeps=sweeps, group=32)
+    sign = (-1.0) ** np.add.outer(np.arange(16), np.arange(64))
+    np.testing.assert_array_equal(q["codes"], np.where(sign > 0, 3, 0))
+    np.testing.assert_allclose(q["m"], -1.0, rtol=1e-13)
+    np.testing.assert_allclose(q["s"], 2.0 / 3.0, rtol=1e-13)
+
+
+def test_checkerboard_is_fixed_point():
+    sign = (-1.0) ** np.add.outer(np.arange(128), np.arange(64))
+    r, c = oracle.normalize(sign, 4)
+    np.testing.assert_array_equal(r, np.ones(128))
+    np.testing.assert_array_equal(c, np.ones(64))
+
+
+@pytest.mark.parametrize("hb", [0, 64])
+def test_power_of_two_token_scaling_is_exact(hb):
+    """Scaling token t by 2^k scales r_t by exactly 2^k and changes nothing else (bit-exact)."""
+    X, _ = _config0_k(1)
+    X = X[:128]
+    X2 = X.copy()
+    X2[5] *= 2.0 ** 7
+    X2[77] *= 2.0 ** -3
+    q1 = oracle.quantize_block(X, hb=hb, sweeps=4)
+    q2 = oracle.quantize_block(X2, hb=hb, sweeps=4)
+    expect_r = q1["r"].copy()
+    expect_r[5] *= 2.0 ** 7
+    expect_r[77] *= 2.0 ** -3
+    np.testing.assert_array_equal(q2["r"], expect_r)
+    np.testing.assert_array_equal(q2["c"], q1["c"])
+    np.testing.assert_array_equal(q2["codes"], q1["codes"])
+    np.testing.assert_array_equal(q2["s"], q1["s"])
+    np.testing.assert_array_equal(q2["m"], q1["m"])
+
+
+def test_zero_rows_and_columns_get_unit_scale():
+    X = np.random.default_rng(2).standard_normal((128, 64))
+    X[3] = 0.0
+    X[:, 10] = 0.0
+    r, c = oracle.normalize(X, 4)
+    assert r[3] == 1.0 and c[10] == 1.0
+    q = oracle.quantize_block(X, hb=0, sweeps=4)
+    assert np.all(q["codes"][3] == 0) and np.all(q["s"][3] == 0.0)
+
+
+def test_zero_sweeps_is_plain_group_rtn():
+    X = np.random.default_rng(4).standard_normal((128, 64))
+    r, c = oracle.normalize(X, 0)
+    assert np.all(r == 1.0) and np.all(c == 1.0)
+
+
+# --------------------------------------------------------------------- codec
+def test_grid_values_round_trip_exactly():
+    """Values on the 2-bit grid {m + k s} with binary16-exact m, s come back exactly."""
+    rng = np.random.default_rng(5)
+    T, D = 128, 64
+    m = rng.integers(-64, 64, size=(T, 2)) / 16.0
+    s = rng.integers(1, 32, size=(T, 2)) / 32.0
+    k = rng.integers(0, 4, size=(T, D))
+    k[:, 0], k[:, 1], k[:, 32], k[:, 33] = 0, 3, 0, 3  # every group spans the full grid
+    X = m.repeat(32, axis=1) + k * s.repeat(32, axis=1)
+    q = oracle.quantize_block(X, hb=0, sweeps=0)
+    np.testing.assert_array_equal(q["codes"], k)
+    rec = oracle.pack_record(q)
+    np.testing.assert_array_equal(oracle.dequantize_record(rec, T, D, hb=0), X)
+
+
+def test_codes_are_the_nearest_level():
+    """Brute force: the code is the nearest of the four levels m + k s (ties excluded)."""
+    X, _ = _config0_k(2)
+    q = oracle.quantize_block(X[:128], hb=64, sweeps=4)
+    Y = q["xrot"] / (q["r"][:, None] * q["c"][None, :])
+    lv = q["m"].repeat(32, axis=1)[..., None] + np.arange(4) * q["s"].repeat(32, axis=1)[..., None]
+    best = np.argmin(np.abs(Y[..., None] - lv), axis=-1)
+    tie = np.abs(q["v"] - np.floor(q["v"]) - 0.5) < 1e-9
+    assert np.array_equal(best[~tie], q["codes"][~tie])
+    assert q["codes"].max() == 3 and q["codes"].min() == 0
+
+
+def test_dequantisation_error_is_at_most_half_a_step():
+    X, _ = _config0_k(3)
+    q = oracle.quantize_block(X[128:], hb=64, sweeps=4)
+    rec = oracle.pack_record(q)
+    u = oracle.unpack_record(rec, 128, 64)
+    Xr_hat = oracle.dequantize_record(rec, 128, 64, hb=64, rotated=True)
+    step = (u["r"][:, None] * u["c"][None, :]) * u["s"].repeat(32, axis=1)
+    # error of RTN with the unrounded scales, plus what binary16 rounding of r, c, s, m may add
+    slack = 4 * 2.0 ** -11 * np.abs(q["xrot"]) + 2 * 2.0 ** -11 * np.abs(
+        u["r"][:, None] * u["c"][None, :] * u["m"].repeat(32, axis=1))
+    assert np.all(np.abs(Xr_hat - q["xrot"]) <= 0.5 * step + slack + 1e-12)
+    # the unrotated dequantisation is the rotated one rotated back
+    np.testing.assert_allclose(oracle.dequantize_record(rec, 128, 64, hb=64), oracle.rotate(Xr_hat, 64), atol=1e-12)
+
+
+def test_binary16_rounding_matches_numpy():
+    rng = np.random.default_rng(6)
+    xs = np.concatenate([
+        rng.standard_normal(4000) * np.exp(rng.uniform(-25, 12, 4000)),
+        [0.0, -0.0, 65504.0, 65519.99, 65520.0, 1e6, -1e6, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -26,
+         2.0 ** -14, 2.0 ** -14 * (1 - 2.0 ** -11), 1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, float("inf")]])
+    for x in xs:
+        assert oracle.f16_bits(x) == int(np.array(x, dtype=np.float64).astype(np.float16).view(np.uint16)), x
+    for bits in list(range(0, 0x7C01, 37)) + [0x8001, 0xBC00, 0x7BFF]:
+        assert oracle.f16_value(bits) == float(np.array(bits, dtype=np.uint16).view(np.float16))
+
+
+def test_record_bit_layout():
+    T, D = 128, 64
+    codes = np.zeros((T, D), dtype=np.uint8)
+    codes[0, :4] = [0, 1, 2, 3]
+    codes[1, 4:8] = [3, 2, 1, 0]
+    q = dict(codes=codes, r=np.full(T, 2.0), c=np.full(D, 0.5), s=np.full((T, 2), 0.25), m=np.full((T, 2), -1.0))
+    rec = oracle.pack_record(q)
+    assert len(rec) == oracle.record_bytes(T, D) == 3456  # 2048 + 1024 + 256 + 128, already 128-aligned
+    assert rec[0] == 0xE4 and rec[1] == 0 and rec[16 + 1] == 0x1B
+    g = np.frombuffer(rec[2048:2048 + 1024].tobytes(), dtype=np.float16).reshape(T, 2, 2)
+    assert np.all(g[..., 0] == 0.25) and np.all(g[..., 1] == -1.0)
+    assert np.all(np.frombuffer(rec[3072:3328].tobytes(), dtype=np.float16) == 2.0)
+    assert np.all(np.frombuffer(rec[3328:3456].tobytes(), dtype=np.float16) == 0.5)
+    assert oracle.record_bytes(128, 128) == 6656 and oracle.record_bytes(128, 96) == 5120
+
+
+# ----------------------------------------------------------------- attention
+def _sdpa(q, K, V, scale):
+    """Library reference: torch scaled_dot_product_attention in fp64, kv heads repeated."""
+    Hq, Hkv = q.shape[0], K.shape[0]
+    rep = Hq // Hkv
+    Kt = torch.from_numpy(np.repeat(K, rep, axis=0))
+    Vt = torch.from_numpy(np.repeat(V, rep, axis=0))
+    qt = torch.from_numpy(q)[:, None, :]
+    o = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt, scale=scale)
+    return o[:, 0, :].numpy()
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(1, 1), (4, 1), (8, 2)])
+def test_attention_brute_force_16_tokens(Hq, Hkv):
+    rng = np.random.default_rng(8)
+    D, L = 64, 16
+    q = rng.standard_normal((Hq, D))
+    K = rng.standard_normal((Hkv, L, D)) * 2
+    V = rng.standard_normal((Hkv, L, D))
+    out = oracle.attention(q, K, V, 1 / math.sqrt(D))
+    np.testing.assert_allclose(out, _sdpa(q, K, V, 1 / math.sqrt(D)), rtol=0, atol=1e-12)
+
+
+def test_gqa_equals_repeated_mha():
+    rng = np.random.default_rng(9)
+    q = rng.standard_normal((8, 32))
+    K = rng.standard_normal((2, 20, 32))
+    V = rng.standard_normal((2, 20, 32))
+    a = oracle.attention(q, K, V, 0.3)
+    b = oracle.attention(q, np.repeat(K, 4, axis=0), np.repeat(V, 4, axis=0), 0.3)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-14)
+
+
+def test_attention_is_rotation_invariant_in_scores():
+    rng = np.random.default_rng(10)
+    q = rng.standard_normal((2, 64))
+    K = rng.standard_normal((1, 30, 64))
+    V = rng.standard_normal((1, 30, 64))
+    a = oracle.attention(q, K, V, 0.125)
+    b = oracle.attention(oracle.rotate(q, 64), oracle.rotate(K, 64), V, 0.125)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("n_tokens", [0, 5, 8, 13, 16])
+def test_decode_from_cache_brute_force(n_tokens):
+    """16-token cache, 8-token blocks: two packed blocks, one block + tail, tail only, empty."""
+    rng = np.random.default_rng(11)
+    T, D, Hkv, Hq = 8, 64, 2, 4
+    Kx = rng.standard_normal((Hkv, 16, D)) * 3
+    Vx = rng.standard_normal((Hkv, 16, D))
+    q = rng.standard_normal((Hq, D))
+    nb = n_tokens // T
+    krec = np.zeros((Hkv, 2, oracle.record_bytes(T, D)), dtype=np.uint8)
+    vrec = np.zeros_like(krec)
+    Khat = np.zeros((Hkv, n_tokens, D))
+    Vhat = np.zeros((Hkv, n_tokens, D))
+    for h in range(Hkv):
+        for b in range(nb):
+            krec[h, b] = oracle.pack_record(oracle.quantize_block(Kx[h, b * T:(b + 1) * T], 64, 4))
+            vrec[h, b] = oracle.pack_record(oracle.quantize_block(Vx[h, b * T:(b + 1) * T], 64, 4))
+            Khat[h, b * T:(b + 1) * T] = oracle.dequantize_record(krec[h, b], T, D, 64)
+            Vhat[h, b * T:(b + 1) * T] = oracle.dequantize_record(vrec[h, b], T, D, 64)
+        Khat[h, nb * T:] = Kx[h, nb * T:n_tokens]
+        Vhat[h, nb * T:] = Vx[h, nb * T:n_tokens]
+    ktail = np.zeros((Hkv, T, D))
+    vtail = np.zeros((Hkv, T, D))
+    ktail[:, :n_tokens - nb * T] = Kx[:, nb * T:n_tokens]
+    vtail[:, :n_tokens - nb * T] = Vx[:, nb * T:n_tokens]
+    out = oracle.decode_from_cache(q, krec, vrec, ktail, vtail, n_tokens, T, 64, 1 / 8)
+    if n_tokens == 0:
+        assert np.all(out == 0)
+    else:
+        np.testing.assert_allclose(out, _sdpa(q, Khat, Vhat, 1 / 8), rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------ threaded bulk
+def test_quantize_many_matches_single_blocks():
+    k, _ = synth.layer_kv(0, 0, 1, 2, 256, 64, n_outliers=2, dtype=torch.bfloat16)
+    raw = k.contiguous().view(torch.int16).numpy().view(np.uint16)
+    recs, used = oracle.quantize_many(raw, "bf16", 128, 64, 64, nthreads=3)
+    assert used == 3 and recs.shape == (4, 3456)
+    kd = k.double().numpy().reshape(4, 128, 64)
+    for u in range(4):
+        np.testing.assert_array_equal(recs[u], oracle.pack_record(oracle.quantize_block(kd[u], 64, 4)))
