@@ -1,0 +1,61 @@
+// kvarn_internal.h -- launch argument blocks passed from the C ABI layer to
+// the kernels (by value, in kernel parameter space).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvarn.h"
+
+namespace kvarn {
+
+struct QuantArgs {
+    const void *k, *v;          // [S][Hkv][num_tokens][D]
+    void *k_records, *v_records;
+    void *k_tail, *v_tail;
+    int32_t *n_tokens;
+    int32_t *status;
+    float *debug_k, *debug_v;
+    int num_tokens, first_block, max_blocks, num_kv_heads, sweeps;
+};
+
+struct AppendArgs {
+    const void *k, *v;          // [S][Hkv][D]
+    void *k_records, *v_records;
+    void *k_tail, *v_tail;
+    int32_t *n_tokens;
+    uint32_t *arrive;
+    int32_t *status;
+    int max_blocks, num_kv_heads, sweeps;
+};
+
+struct DequantArgs {
+    const void *k_records, *v_records;
+    float *k_out, *v_out;
+    int first_block, num_blocks, max_blocks, rotated;
+};
+
+struct DecodeArgs {
+    const void *q;              // [S][Hq][D]
+    const void *k_records, *v_records;
+    const void *k_tail, *v_tail;
+    const int32_t *n_tokens;
+    int32_t *status;
+    float *out;                 // [S][Hq][D]
+    float *partials;            // [S*Hkv][nsplit+1][grp][D+2]
+    uint32_t *tickets;          // [S*Hkv]
+    float scale_log2;           // softmax scale * log2(e)
+    int num_kv_heads, grp, max_blocks, max_tokens;
+    int nsplit, blocks_per_split;
+};
+
+cudaError_t run_quantize(const kvarn_config &c, const QuantArgs &a, cudaStream_t st);
+cudaError_t run_append(const kvarn_config &c, const AppendArgs &a, cudaStream_t st);
+cudaError_t run_dequantize(const kvarn_config &c, const DequantArgs &a, cudaStream_t st);
+cudaError_t run_decode(const kvarn_config &c, const DecodeArgs &a, cudaStream_t st);
+cudaError_t run_set_length(int32_t *n_tokens, int num_seqs, int value, cudaStream_t st);
+
+// Largest split count the decode workspace is sized for.
+constexpr int kMaxSplits = 64;
+
+}  // namespace kvarn

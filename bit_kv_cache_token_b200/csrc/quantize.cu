@@ -1,0 +1,166 @@
+// quantize.cu -- bulk quantisation (prefill) and append-with-quantise kernels.
+#include "kvarn_internal.h"
+#include "quantize_block.cuh"
+
+namespace kvarn {
+
+// One CTA per (sequence, kv head, block) and per tensor (blockIdx.y: 0 = K,
+// 1 = V).  Block index nb (one past the full blocks) copies the ragged tail.
+template <int D, int HB, typename Tin>
+__global__ void __launch_bounds__(D, 2)
+quantize_blocks_kernel(QuantArgs a)
+{
+    __shared__ QuantSmem<D> sm;
+    const int nb = a.num_tokens / kBlockTokens;
+    const int rem = a.num_tokens % kBlockTokens;
+    const int nbx = nb + (rem > 0 ? 1 : 0);
+    const int b = blockIdx.x % nbx;
+    const int sh = blockIdx.x / nbx;  // s * Hkv + h
+    const int tensor = blockIdx.y;
+    const Tin *src = static_cast<const Tin *>(tensor ? a.v : a.k) +
+                     (size_t)sh * a.num_tokens * D + (size_t)b * kBlockTokens * D;
+
+    if (b == 0 && tensor == 0 && (sh % a.num_kv_heads) == 0 && threadIdx.x == 0)
+        a.n_tokens[sh / a.num_kv_heads] = a.first_block * kBlockTokens + a.num_tokens;
+
+    if (b == nb) {  // residual tail: copied as given, unrotated
+        Tin *tail = static_cast<Tin *>(tensor ? a.v_tail : a.k_tail) + (size_t)sh * kBlockTokens * D;
+        copy_elems(tail, src, rem * D, threadIdx.x, D);
+        return;
+    }
+    float2 X[4][16];
+    load_block<D>(src, X);
+    const size_t slot = (size_t)sh * a.max_blocks + a.first_block + b;
+    unsigned char *rec = static_cast<unsigned char *>(tensor ? a.v_records : a.k_records) +
+                         slot * Record<D>::kBytes;
+    float *dbg = tensor ? a.debug_v : a.debug_k;
+    if (dbg) dbg += ((size_t)sh * nb + b) * (kBlockTokens + D + 2 * kBlockTokens * (D / kGroup));
+    quantize_block<D, HB>(X, sm, a.sweeps, rec, dbg, a.status);
+}
+
+// One CTA per (sequence, kv head) and per tensor.  The token goes into tail
+// slot n % T; if that completes the tail, the CTA quantises the tail into
+// record n / T.  The last CTA of a sequence to finish advances n_tokens[s]
+// (arrival counter, no waiting).
+template <int D, int HB, typename Tin>
+__global__ void __launch_bounds__(D, 2)
+append_kernel(AppendArgs a)
+{
+    __shared__ QuantSmem<D> sm;
+    __shared__ int s_n;
+    const int sh = blockIdx.x;  // s * Hkv + h
+    const int s = sh / a.num_kv_heads;
+    const int tensor = blockIdx.y;
+    if (threadIdx.x == 0) s_n = *reinterpret_cast<volatile int32_t *>(a.n_tokens + s);
+    __syncthreads();
+    const int n = s_n;
+    const int pos = n % kBlockTokens, blk = n / kBlockTokens;
+    const bool fills = pos == kBlockTokens - 1;
+    const bool full = fills && blk >= a.max_blocks;
+
+    if (!full) {
+        Tin *tail = static_cast<Tin *>(tensor ? a.v_tail : a.k_tail) + (size_t)sh * kBlockTokens * D;
+        const Tin *tok = static_cast<const Tin *>(tensor ? a.v : a.k) + (size_t)sh * D;
+        copy_elems(tail + (size_t)pos * D, tok, D, threadIdx.x, D);
+        if (fills) {
+            __syncthreads();  // the new row is visible to the whole CTA
+            float2 X[4][16];
+            load_block<D>(tail, X);
+            unsigned char *rec = static_cast<unsigned char *>(tensor ? a.v_records : a.k_records) +
+                                 ((size_t)sh * a.max_blocks + blk) * Record<D>::kBytes;
+            quantize_block<D, HB>(X, sm, a.sweeps, rec, nullptr, a.status);
+        }
+    } else if (threadIdx.x == 0 && tensor == 0 && (sh % a.num_kv_heads) == 0) {
+        status_or(a.status, KVARN_STATUS_CAPACITY);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(a.arrive + s, 1u);
+        if (prev == 2u * a.num_kv_heads - 1u) {
+            __threadfence();
+            a.arrive[s] = 0u;
+            if (!full) a.n_tokens[s] = n + 1;
+        }
+    }
+}
+
+template <int D, int HB, typename Tin>
+static cudaError_t launch_quant(const QuantArgs &a, int S, int Hkv, cudaStream_t st)
+{
+    const int nb = a.num_tokens / kBlockTokens;
+    const int nbx = nb + (a.num_tokens % kBlockTokens ? 1 : 0);
+    if (nbx == 0) return cudaSuccess;
+    dim3 grid((unsigned)(S * Hkv * nbx), 2);
+    quantize_blocks_kernel<D, HB, Tin><<<grid, D, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <int D, int HB, typename Tin>
+static cudaError_t launch_append(const AppendArgs &a, int S, int Hkv, cudaStream_t st)
+{
+    dim3 grid((unsigned)(S * Hkv), 2);
+    append_kernel<D, HB, Tin><<<grid, D, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+// ---- dispatch over (D, Hadamard block, dtype) ---------------------------
+#define KVARN_DISPATCH_HB(D, HB, FN, ...)                                            \
+    (dtype == KVARN_BF16 ? FN<D, HB, __nv_bfloat16>(__VA_ARGS__) : FN<D, HB, float>(__VA_ARGS__))
+
+template <int D>
+static cudaError_t dispatch_quant(int hb, int dtype, const QuantArgs &a, int S, int Hkv, cudaStream_t st)
+{
+    switch (hb) {
+    case 0: return KVARN_DISPATCH_HB(D, 0, launch_quant, a, S, Hkv, st);
+    case 32: return KVARN_DISPATCH_HB(D, 32, launch_quant, a, S, Hkv, st);
+    case 64: if constexpr (D % 64 == 0) return KVARN_DISPATCH_HB(D, 64, launch_quant, a, S, Hkv, st); break;
+    case 128: if constexpr (D % 128 == 0) return KVARN_DISPATCH_HB(D, 128, launch_quant, a, S, Hkv, st); break;
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <int D>
+static cudaError_t dispatch_append(int hb, int dtype, const AppendArgs &a, int S, int Hkv, cudaStream_t st)
+{
+    switch (hb) {
+    case 0: return KVARN_DISPATCH_HB(D, 0, launch_append, a, S, Hkv, st);
+    case 32: return KVARN_DISPATCH_HB(D, 32, launch_append, a, S, Hkv, st);
+    case 64: if constexpr (D % 64 == 0) return KVARN_DISPATCH_HB(D, 64, launch_append, a, S, Hkv, st); break;
+    case 128: if constexpr (D % 128 == 0) return KVARN_DISPATCH_HB(D, 128, launch_append, a, S, Hkv, st); break;
+    }
+    return cudaErrorInvalidValue;
+}
+
+__global__ void set_length_kernel(int32_t *n_tokens, int num_seqs, int value)
+{
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < num_seqs; i += gridDim.x * blockDim.x) n_tokens[i] = value;
+}
+
+cudaError_t run_set_length(int32_t *n_tokens, int num_seqs, int value, cudaStream_t st)
+{
+    set_length_kernel<<<(num_seqs + 255) / 256, 256, 0, st>>>(n_tokens, num_seqs, value);
+    return cudaGetLastError();
+}
+
+cudaError_t run_quantize(const kvarn_config &c, const QuantArgs &a, cudaStream_t st)
+{
+    switch (c.head_dim) {
+    case 64: return dispatch_quant<64>(c.hadamard, c.dtype, a, c.num_seqs, c.num_kv_heads, st);
+    case 96: return dispatch_quant<96>(c.hadamard, c.dtype, a, c.num_seqs, c.num_kv_heads, st);
+    case 128: return dispatch_quant<128>(c.hadamard, c.dtype, a, c.num_seqs, c.num_kv_heads, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t run_append(const kvarn_config &c, const AppendArgs &a, cudaStream_t st)
+{
+    switch (c.head_dim) {
+    case 64: return dispatch_append<64>(c.hadamard, c.dtype, a, c.num_seqs, c.num_kv_heads, st);
+    case 96: return dispatch_append<96>(c.hadamard, c.dtype, a, c.num_seqs, c.num_kv_heads, st);
+    case 128: return dispatch_append<128>(c.hadamard, c.dtype, a, c.num_seqs, c.num_kv_heads, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace kvarn
