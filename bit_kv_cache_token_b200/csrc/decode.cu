@@ -1,24 +1,35 @@
-// decode.cu -- split-K single-token decode attention over the packed cache.
+// decode.cu -- single-token decode attention over the packed 2-bit cache.
 //
-// KVarN decode (abstract: attention over the 2-bit cache during long-horizon
+// KVarN decode (abstract: attention over the 2-bit cache in long-horizon
 // decoding; rndamp.com article, "Numbers": the second scale is fused into the
-// dequantisation kernel).  The keys are stored rotated, so the query is
-// rotated once (normalised Hadamard, per Hadamard block) and the scores are
-// taken in the rotated basis, where q . k is unchanged.  With
-// k_rot[t][d] = r_t c_d (s_{t,g} code + m_{t,g}):
+// dequantisation kernel).  Keys are stored rotated, so the query is rotated
+// once and scores are taken in the rotated basis, where q . k is unchanged.
+// With k_rot[t][d] = r_t c_d (s_{t,g} code + m_{t,g}):
 //   score_t = r_t * sum_g ( s_{t,g} * sum_{d in g} q'_d code_{t,d} + m_{t,g} Q_g ),
-//   q'_d = q_rot,d * c_d * scale,   Q_g = sum_{d in g} q'_d,
-// so c^K folds into the query once per block and r^K, s^K, m^K into one FMA
-// per (token, group).  For V, with p_t the softmax weight:
-//   o_rot,d += c^V_d * sum_t ( p_t r^V_t s^V_{t,g} code_{t,d} + p_t r^V_t m^V_{t,g} ).
+//   q'_d = q_rot,d * c^K_d * scale,  Q_g = sum_{d in g} q'_d;
+// and with p_t the softmax weight,
+//   o_rot,d = c^V_d * sum_t ( p_t r^V_t s^V_{t,g} code_{t,d} + p_t r^V_t m^V_{t,g} ).
 // The residual tail (unrotated, input dtype) is attended with the unrotated
-// query in its own split; the combine merges all splits with log-sum-exp
-// weights, rotates the block part back and adds the tail part.
+// query; the combine merges all partials with log-sum-exp weights, rotates
+// the block part back and adds the tail part.
 //
-// Grid: (S * Hkv, nsplit + 1); split nsplit is the tail.  The query heads of
-// one kv head (GQA group) share every code load.  The last CTA of a
-// (sequence, kv head) to finish, found with an atomic ticket, combines.  No
-// CTA ever waits for another.
+// B200 mapping.  One warp streams a contiguous range of 128-token blocks of
+// one (sequence, kv head) with its own online softmax; the records reach
+// shared memory by cp.async.bulk (TMA) into a two-stage ring guarded by
+// mbarriers.  Both contractions run on tensor cores (mma.sync m16n8k16, fp16
+// in, fp32 accumulate):
+//   scores: A = q' (rows: query heads; hi/lo fp16 split in rows 0-7 / 8-15),
+//           B = K codes (k = channels, n = 8 tokens);
+//   P V:    A = p r s (rows: heads, hi/lo), B = V codes (k = tokens, n = 8 channels).
+// A 2-bit code becomes an exact fp16 operand with a single AND: the record
+// stores every code in a 32-bit word at bit 16*half + 2*pos (see kvarn.h),
+// so masking with 0x00030003 << 2*(pos%4) yields the pair as fp16 subnormals
+// c * 2^(2*(pos%4) - 24).  The 2^-(2*(pos%4)) part is folded into the other
+// operand (it depends only on the contracted index) and the remaining 2^-18
+// into the scales.  When the GQA group has fewer than 8 heads, the spare rows
+// carry copies of the heads working on other channel groups, so every lane
+// does useful work.  The last warp of a (sequence, kv head) to finish,
+// found with an atomic ticket, combines; no warp ever waits for another.
 #include <math.h>
 
 #include "kvarn_common.cuh"
@@ -26,342 +37,590 @@
 
 namespace kvarn {
 
-constexpr int kDecThreads = 128;
+constexpr int kDecWarps = 6;
+constexpr float kTwo18 = 262144.f;          // 2^18
+constexpr float kTwoM18 = 1.f / 262144.f;   // 2^-18
+constexpr long long kWaitLimit = 1LL << 26; // bounded mbarrier polling
 
 template <int D, int GRP>
-struct DecSmem {
-    unsigned char krec[Record<D>::kBytes];
-    unsigned char vrec[Record<D>::kBytes];
-    float qrot[GRP][D];          // rotated (blocks) or plain (tail) query, pre-scaled
-    float qp[GRP][D];            // q' for the current block
-    float Qg[GRP][D / kGroup];
-    float pw[kBlockTokens][D / kGroup][GRP];  // p_t r_t s_{t,g} per head
-    float pr[kBlockTokens][GRP];              // p_t r_t per head
-    float bias[GRP][D / kGroup];
-    float red[kDecThreads / 32][GRP];
-    float mnew[GRP], alpha[GRP], lsum[GRP];
-    int last;
+struct alignas(128) DecWarpSmem {
+    unsigned char rec[2][2][Record<D>::kBytes];  // [stage][K, V]
+    float scr[(D / kGroup) * kBlockTokens + kBlockTokens + D];
+    float qbuf[GRP][D];
+    unsigned long long mbar[2];
 };
 
-__device__ __forceinline__ float code_f(uint32_t word, int i)
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
-    // (word >> 2i) & 3 as an exact float: OR the code into the mantissa of 2^23
-    return __uint_as_float(0x4B000000u | ((word >> (2 * i)) & 3u)) - 8388608.f;
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// In-place normalised Walsh-Hadamard transform of nvec vectors of length D
-// in shared memory, Hadamard block hb (0 = none).  All threads call it.
-__device__ void smem_fwht(float *x, int nvec, int D, int hb)
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
 {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// fp32 pair -> (hi, lo) fp16 pairs with hi + lo = x to about 2^-22 relative.
+__device__ __forceinline__ void split_hilo(float x, float y, uint32_t &hi, uint32_t &lo)
+{
+    const __half2 h = __floats2half2_rn(x, y);
+    const float2 hf = __half22float2(h);
+    const __half2 l = __floats2half2_rn(x - hf.x, y - hf.y);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+// Two codes at position pos of word w as an fp16 pair (subnormal values).
+__device__ __forceinline__ uint32_t code_pair(uint32_t w, uint32_t w8, int pos)
+{
+    return pos < 4 ? (w & (0x00030003u << (2 * pos))) : (w8 & (0x00030003u << (2 * (pos - 4))));
+}
+
+__device__ __forceinline__ void mbar_init(unsigned long long *bar)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(bar)));
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+
+// Lane 0 only: stage both records of block b (K then V) into stage buffers.
+__device__ __forceinline__ void issue_block(unsigned long long *bar, unsigned char *kdst, unsigned char *vdst,
+                                            const unsigned char *ksrc, const unsigned char *vsrc, uint32_t bytes)
+{
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(2 * bytes)
+                 : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                     smem_u32(kdst)),
+                 "l"(ksrc), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                     smem_u32(vdst)),
+                 "l"(vsrc), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Bounded wait for phase `parity` of an mbarrier; false if the limit ran out.
+__device__ __forceinline__ bool mbar_wait(unsigned long long *bar, uint32_t parity)
+{
+    for (long long i = 0; i < kWaitLimit; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+            : "=r"(done)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+// Normalised Walsh-Hadamard transform (block hb, 0 = none) of nvec rows of
+// length D in shared memory, by one warp.
+template <int D>
+__device__ void warp_fwht(float *x, int nvec, int hb)
+{
+    const int lane = threadIdx.x & 31;
     if (hb == 0) return;
     for (int h = 1; h < hb; h <<= 1) {
-        for (int idx = threadIdx.x; idx < nvec * D / 2; idx += blockDim.x) {
+        for (int idx = lane; idx < nvec * D / 2; idx += 32) {
             const int v = idx / (D / 2), p = idx % (D / 2);
-            // p-th pair of this stage: index with bit h cleared
             const int lo = (p / h) * 2 * h + (p % h);
             float *row = x + v * D;
             const float a = row[lo], b = row[lo + h];
             row[lo] = a + b;
             row[lo + h] = a - b;
         }
-        __syncthreads();
+        __syncwarp();
     }
     const float nrm = rsqrtf((float)hb);
-    for (int idx = threadIdx.x; idx < nvec * D; idx += blockDim.x) x[idx] *= nrm;
-    __syncthreads();
-}
-
-template <int GRP>
-__device__ __forceinline__ void block_reduce(float (&v)[GRP], float (*red)[GRP], bool is_max)
-{
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-#pragma unroll
-    for (int h = 0; h < GRP; ++h) {
-        float x = v[h];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float y = __shfl_xor_sync(0xffffffffu, x, o);
-            x = is_max ? fmaxf(x, y) : x + y;
-        }
-        if (l == 0) red[w][h] = x;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < GRP; ++h) {
-        float x = red[0][h];
-#pragma unroll
-        for (int ww = 1; ww < kDecThreads / 32; ++ww) x = is_max ? fmaxf(x, red[ww][h]) : x + red[ww][h];
-        v[h] = x;
-    }
-    __syncthreads();
+    for (int idx = lane; idx < nvec * D; idx += 32) x[idx] *= nrm;
+    __syncwarp();
 }
 
 template <int D, int GRP, typename Tin>
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kDecWarps * 32, 1)
 decode_kernel(DecodeArgs a, int hb)
 {
     using R = Record<D>;
-    constexpr int NG = D / kGroup;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    DecSmem<D, GRP> &sm = *reinterpret_cast<DecSmem<D, GRP> *>(smem_raw);
-    const int tid = threadIdx.x;
-    const int sh = blockIdx.x, split = blockIdx.y;
-    const int s = sh / a.num_kv_heads;
-    const bool is_tail = split == a.nsplit;
+    constexpr int NG = D / kGroup;          // channel groups
+    constexpr int NKT = D / 16;             // k-tiles of the score MMA
+    constexpr int NNT = D / 8;              // n-tiles of the P V MMA
+    constexpr int C = 8 / GRP;              // head copies in the 8 MMA rows
+    constexpr int SETS = (NG + C - 1) / C;  // groups handled per copy
+    constexpr int KW = D / 32;              // K code words per (16-token unit, lane)
+    constexpr int F = D / 64;
+
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    DecWarpSmem<D, GRP> &sm = reinterpret_cast<DecWarpSmem<D, GRP> *>(smem_raw)[warp];
+    const int item = blockIdx.x * kDecWarps + warp;
+    const int nitems = a.num_units * a.nsplit;
+    if (item >= nitems) return;
+    const int unit = item / a.nsplit, split = item % a.nsplit;
+    const int s = unit / a.num_kv_heads;
+    const int gl = lane >> 2, tig = lane & 3;  // mma groupID, thread in group
+    const int copy = gl / GRP, h = gl % GRP;
 
     int n = a.n_tokens[s];
     if (n > a.max_tokens) {
-        if (tid == 0 && split == 0) status_or(a.status, KVARN_STATUS_LENGTH);
+        if (lane == 0 && split == 0) status_or(a.status, KVARN_STATUS_LENGTH);
         n = a.max_tokens;
     }
+    if (n < 0) n = 0;
     const int nblk = n / kBlockTokens;
     const int ntail = n - nblk * kBlockTokens;
+    const int b0 = split * a.blocks_per_split;
+    const int b1 = min(b0 + a.blocks_per_split, nblk);
 
-    // query of the GQA group, times softmax scale * log2(e)
-    const Tin *q = static_cast<const Tin *>(a.q) + ((size_t)sh * GRP) * D;
-    for (int idx = tid; idx < GRP * D; idx += kDecThreads)
-        (&sm.qrot[0][0])[idx] = In<Tin>::load1(q + idx) * a.scale_log2;
-    __syncthreads();
-    if (!is_tail) smem_fwht(&sm.qrot[0][0], GRP, D, hb);
+    // ---- rotated query of this GQA group, scaled by softmax scale * log2(e)
+    const Tin *qg = static_cast<const Tin *>(a.q) + (size_t)unit * GRP * D;
+    for (int i = lane; i < GRP * D; i += 32) (&sm.qbuf[0][0])[i] = In<Tin>::load1(qg + i) * a.scale_log2;
+    __syncwarp();
+    warp_fwht<D>(&sm.qbuf[0][0], GRP, hb);
+    float qreg[NKT][4];  // q_rot at channels 16kt + 2tig + {0, 1, 8, 9}
+#pragma unroll
+    for (int kt = 0; kt < NKT; ++kt) {
+        const int k = 16 * kt + 2 * tig;
+        qreg[kt][0] = sm.qbuf[h][k];
+        qreg[kt][1] = sm.qbuf[h][k + 1];
+        qreg[kt][2] = sm.qbuf[h][k + 8];
+        qreg[kt][3] = sm.qbuf[h][k + 9];
+    }
 
-    float m_run[GRP], l_run[GRP], acc[GRP];
+    float m_run = -INFINITY, l_run = 0.f;
+    float2 orun[NNT];
 #pragma unroll
-    for (int h = 0; h < GRP; ++h) { m_run[h] = -INFINITY; l_run[h] = 0.f; acc[h] = 0.f; }
+    for (int i = 0; i < NNT; ++i) orun[i] = f2(0.f, 0.f);
+    int failed_at = -1;  // block index whose copy did not arrive in time
 
-    if (!is_tail) {
-        const int b0 = split * a.blocks_per_split;
-        const int b1 = min(b0 + a.blocks_per_split, nblk);
-        const unsigned char *kbase = static_cast<const unsigned char *>(a.k_records) + (size_t)sh * a.max_blocks * R::kBytes;
-        const unsigned char *vbase = static_cast<const unsigned char *>(a.v_records) + (size_t)sh * a.max_blocks * R::kBytes;
-        for (int b = b0; b < b1; ++b) {
-            // -- stage both records in shared memory (coalesced 16-byte loads)
-            const uint4 *ks = reinterpret_cast<const uint4 *>(kbase + (size_t)b * R::kBytes);
-            const uint4 *vs = reinterpret_cast<const uint4 *>(vbase + (size_t)b * R::kBytes);
-            for (int i = tid; i < R::kBytes / 16; i += kDecThreads) {
-                reinterpret_cast<uint4 *>(sm.krec)[i] = __ldcs(ks + i);
-                reinterpret_cast<uint4 *>(sm.vrec)[i] = __ldcs(vs + i);
+    const unsigned char *kbase = static_cast<const unsigned char *>(a.k_records) + (size_t)unit * a.max_blocks * R::kBytes;
+    const unsigned char *vbase = static_cast<const unsigned char *>(a.v_records) + (size_t)unit * a.max_blocks * R::kBytes;
+    if (lane == 0) {
+        mbar_init(&sm.mbar[0]);
+        mbar_init(&sm.mbar[1]);
+    }
+    __syncwarp();
+    if (lane == 0) {
+        for (int i = 0; i < 2 && b0 + i < b1; ++i)
+            issue_block(&sm.mbar[i], sm.rec[i][0], sm.rec[i][1], kbase + (size_t)(b0 + i) * R::kBytes,
+                        vbase + (size_t)(b0 + i) * R::kBytes, R::kBytes);
+    }
+
+    for (int b = b0; b < b1; ++b) {
+        const int i = b - b0, stage = i & 1;
+        if (!mbar_wait(&sm.mbar[stage], (i >> 1) & 1)) { failed_at = i; break; }
+        const unsigned char *krec = sm.rec[stage][0];
+        const unsigned char *vrec = sm.rec[stage][1];
+        float *scr = sm.scr;
+
+        // ---- K scales to fp32: sK[g][t] = s * 2^18, rK[t], cK[d]
+        {
+            const __half *sh = reinterpret_cast<const __half *>(krec + R::kSOff);
+            for (int idx = lane; idx < NG * kBlockTokens; idx += 32) {
+                const int t = idx / NG, g = idx % NG;
+                scr[g * kBlockTokens + t] = __half2float(sh[idx]) * kTwo18;
             }
-            __syncthreads();
-            // -- q' = q_rot * c^K and its group sums
-            const __half *cK = reinterpret_cast<const __half *>(sm.krec + R::kCOff);
-            for (int idx = tid; idx < GRP * D; idx += kDecThreads) {
-                const int d = idx % D;
-                (&sm.qp[0][0])[idx] = (&sm.qrot[0][0])[idx] * __half2float(cK[d]);
+            const __half *rh = reinterpret_cast<const __half *>(krec + R::kROff);
+            for (int t = lane; t < kBlockTokens; t += 32) scr[NG * kBlockTokens + t] = __half2float(rh[t]);
+            const __half *ch = reinterpret_cast<const __half *>(krec + R::kCOff);
+            for (int d = lane; d < D; d += 32) scr[(NG + 1) * kBlockTokens + d] = __half2float(ch[d]);
+        }
+        __syncwarp();
+        const float *sK = scr, *rK = scr + NG * kBlockTokens, *cK = scr + (NG + 1) * kBlockTokens;
+
+        // ---- q' fragments (hi/lo rows) and the per-group sums Q_g
+        uint32_t Aq[NKT][4];
+        float Qg[NG];
+#pragma unroll
+        for (int g = 0; g < NG; ++g) Qg[g] = 0.f;
+#pragma unroll
+        for (int kt = 0; kt < NKT; ++kt) {
+            const int k = 16 * kt + 2 * tig;
+            const float v0 = qreg[kt][0] * cK[k], v1 = qreg[kt][1] * cK[k + 1];
+            const float v2 = qreg[kt][2] * cK[k + 8], v3 = qreg[kt][3] * cK[k + 9];
+            Qg[kt / 2] += (v0 + v1) + (v2 + v3);
+            const int g = kt / 2;
+            const bool mine = (g % C) == copy;
+            // fold the code scale 2^(2*(q%4)) of channel block q = k/8 into q'
+            const float e0 = (kt & 1) ? 4.f : 64.f;   // q = 2kt
+            const float e1 = (kt & 1) ? 1.f : 16.f;   // q = 2kt + 1
+            if (mine) {
+                split_hilo(v0 * e0, v1 * e0, Aq[kt][0], Aq[kt][1]);
+                split_hilo(v2 * e1, v3 * e1, Aq[kt][2], Aq[kt][3]);
+            } else {
+                Aq[kt][0] = Aq[kt][1] = Aq[kt][2] = Aq[kt][3] = 0u;
             }
-            __syncthreads();
-            if (tid < GRP * NG) {
-                const int h = tid / NG, g = tid % NG;
-                float t = 0.f;
-#pragma unroll 8
-                for (int i = 0; i < kGroup; ++i) t += sm.qp[h][g * kGroup + i];
-                sm.Qg[h][g] = t;
+        }
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            Qg[g] += __shfl_xor_sync(0xffffffffu, Qg[g], 1);
+            Qg[g] += __shfl_xor_sync(0xffffffffu, Qg[g], 2);
+        }
+        uint32_t AM[4] = {0u, 0u, 0u, 0u};  // M-term: rows = heads (copy 0), k = group
+        {
+            float q0 = 0.f, q1 = 0.f;
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+                if (g == 2 * tig) q0 = Qg[g];
+                if (g == 2 * tig + 1) q1 = Qg[g];
             }
-            __syncthreads();
-            // -- scores, one token per thread
-            const int t = tid;
-            float sc[GRP];
-            {
-                const float rK = __half2float(reinterpret_cast<const __half *>(sm.krec + R::kROff)[t]);
+            if (copy == 0) split_hilo(q0, q1, AM[0], AM[1]);
+        }
+
+        // ---- scores, 8 tokens per n-tile
+        float2 sc[16];
 #pragma unroll
-                for (int h = 0; h < GRP; ++h) sc[h] = 0.f;
+        for (int u = 0; u < 8; ++u) {
+            uint32_t kw[KW], kw8[KW];
+            const uint32_t *wp = reinterpret_cast<const uint32_t *>(krec) + (u * 32 + lane) * KW;
 #pragma unroll
-                for (int g = 0; g < NG; ++g) {
-                    const __half2 gp = reinterpret_cast<const __half2 *>(sm.krec + R::kGpOff)[t * NG + g];
-                    const float sK = __low2float(gp), mK = __high2float(gp);
-                    const uint2 cw = *reinterpret_cast<const uint2 *>(sm.krec + t * (D / 4) + 8 * g);
-                    float dot[GRP];
+            for (int w = 0; w < KW; ++w) {
+                kw[w] = wp[w];
+                kw8[w] = kw[w] >> 8;
+            }
 #pragma unroll
-                    for (int h = 0; h < GRP; ++h) dot[h] = 0.f;
+            for (int ntl = 0; ntl < 2; ++ntl) {
+                const int nt8 = 2 * u + ntl;
+                float acc[SETS][4];
 #pragma unroll
-                    for (int i = 0; i < kGroup; ++i) {
-                        const float c = code_f(i < 16 ? cw.x : cw.y, i & 15);
+                for (int st = 0; st < SETS; ++st) acc[st][0] = acc[st][1] = acc[st][2] = acc[st][3] = 0.f;
 #pragma unroll
-                        for (int h = 0; h < GRP; ++h) dot[h] = fmaf(sm.qp[h][g * kGroup + i], c, dot[h]);
+                for (int kt = 0; kt < NKT; ++kt) {
+                    uint32_t bb[2];
+#pragma unroll
+                    for (int cs = 0; cs < 2; ++cs) {
+                        const int q = 2 * kt + cs;
+                        int word, pos;
+                        if (q < 8 * F) { word = ntl * F + q / 8; pos = q % 8; }
+                        else { word = 2 * F; pos = q - 8 * F + 4 * ntl; }
+                        bb[cs] = code_pair(kw[word], kw8[word], pos);
                     }
+                    mma16816(acc[(kt / 2) / C], Aq[kt], bb[0], bb[1]);
+                }
+                float accM[4] = {0.f, 0.f, 0.f, 0.f};
+                {
+                    const int t = 8 * nt8 + gl;
+                    const __half *mh = reinterpret_cast<const __half *>(krec + R::kMOff) + t * NG;
+                    const __half m0 = (2 * tig < NG) ? mh[2 * tig] : __float2half(0.f);
+                    const __half m1 = (2 * tig + 1 < NG) ? mh[2 * tig + 1] : __float2half(0.f);
+                    __half2 mp = __halves2half2(m0, m1);
+                    mma16816(accM, AM, *reinterpret_cast<uint32_t *>(&mp), 0u);
+                }
+                const int t0 = 8 * nt8 + 2 * tig;
+                float2 sum = f2(accM[0] + accM[2], accM[1] + accM[3]);
 #pragma unroll
-                    for (int h = 0; h < GRP; ++h) sc[h] += fmaf(sK, dot[h], mK * sm.Qg[h][g]);
+                for (int st = 0; st < SETS; ++st) {
+                    const int g = st * C + copy;
+                    if (g < NG) {
+                        const float2 P = f2(acc[st][0] + acc[st][2], acc[st][1] + acc[st][3]);
+                        const float2 sp = *reinterpret_cast<const float2 *>(sK + g * kBlockTokens + t0);
+                        sum = __ffma2_rn(P, sp, sum);
+                    }
                 }
 #pragma unroll
-                for (int h = 0; h < GRP; ++h) sc[h] *= rK;
-            }
-            // -- online softmax over this block
-            float bm[GRP];
-#pragma unroll
-            for (int h = 0; h < GRP; ++h) bm[h] = sc[h];
-            block_reduce<GRP>(bm, sm.red, true);
-            float p[GRP], ps[GRP];
-#pragma unroll
-            for (int h = 0; h < GRP; ++h) {
-                const float mn = fmaxf(m_run[h], bm[h]);
-                p[h] = exp2f(sc[h] - mn);
-                ps[h] = p[h];
-            }
-            block_reduce<GRP>(ps, sm.red, false);
-            {
-                const float rV = __half2float(reinterpret_cast<const __half *>(sm.vrec + R::kROff)[t]);
-#pragma unroll
-                for (int h = 0; h < GRP; ++h) sm.pr[t][h] = p[h] * rV;
-#pragma unroll
-                for (int g = 0; g < NG; ++g) {
-                    const __half2 gp = reinterpret_cast<const __half2 *>(sm.vrec + R::kGpOff)[t * NG + g];
-                    const float sV = __low2float(gp);
-#pragma unroll
-                    for (int h = 0; h < GRP; ++h) sm.pw[t][g][h] = p[h] * rV * sV;
+                for (int cb = 1; cb < C; cb <<= 1) {
+                    sum.x += __shfl_xor_sync(0xffffffffu, sum.x, 4 * GRP * cb);
+                    sum.y += __shfl_xor_sync(0xffffffffu, sum.y, 4 * GRP * cb);
                 }
-            }
-#pragma unroll
-            for (int h = 0; h < GRP; ++h) {
-                const float mn = fmaxf(m_run[h], bm[h]);
-                const float al = exp2f(m_run[h] - mn);
-                l_run[h] = l_run[h] * al + ps[h];
-                m_run[h] = mn;
-                if (tid == 0) sm.alpha[h] = al;
-            }
-            __syncthreads();
-            if (tid < GRP * NG) {  // bias_{h,g} = sum_t p_t r_t m^V_{t,g}
-                const int h = tid / NG, g = tid % NG;
-                float bsum = 0.f;
-                for (int tt = 0; tt < kBlockTokens; ++tt) {
-                    const __half2 gp = reinterpret_cast<const __half2 *>(sm.vrec + R::kGpOff)[tt * NG + g];
-                    bsum = fmaf(sm.pr[tt][h], __high2float(gp), bsum);
-                }
-                sm.bias[h][g] = bsum;
-            }
-            __syncthreads();
-            // -- P V, one channel per thread
-            if (tid < D) {
-                const int d = tid, g = d / kGroup;
-                const float cV = __half2float(reinterpret_cast<const __half *>(sm.vrec + R::kCOff)[d]);
-                float pv[GRP];
-#pragma unroll
-                for (int h = 0; h < GRP; ++h) pv[h] = sm.bias[h][g];
-#pragma unroll 4
-                for (int tt = 0; tt < kBlockTokens; ++tt) {
-                    const uint32_t byte = sm.vrec[tt * (D / 4) + d / 4];
-                    const float c = code_f(byte, d & 3);
-#pragma unroll
-                    for (int h = 0; h < GRP; ++h) pv[h] = fmaf(sm.pw[tt][g][h], c, pv[h]);
-                }
-#pragma unroll
-                for (int h = 0; h < GRP; ++h) acc[h] = fmaf(acc[h], sm.alpha[h], cV * pv[h]);
-            }
-            __syncthreads();
-        }
-    } else if (ntail > 0) {
-        // -- residual tail: unrotated query against the stored tokens
-        const Tin *kt = static_cast<const Tin *>(a.k_tail) + (size_t)sh * kBlockTokens * D;
-        const Tin *vt = static_cast<const Tin *>(a.v_tail) + (size_t)sh * kBlockTokens * D;
-        const int t = tid;
-        float sc[GRP];
-#pragma unroll
-        for (int h = 0; h < GRP; ++h) sc[h] = -INFINITY;
-        if (t < ntail) {
-#pragma unroll
-            for (int h = 0; h < GRP; ++h) sc[h] = 0.f;
-            for (int d = 0; d < D; ++d) {
-                const float kv = In<Tin>::load1(kt + (size_t)t * D + d);
-#pragma unroll
-                for (int h = 0; h < GRP; ++h) sc[h] = fmaf(sm.qrot[h][d], kv, sc[h]);
+                sc[nt8] = __fmul2_rn(sum, *reinterpret_cast<const float2 *>(rK + t0));
             }
         }
-        float bm[GRP];
+
+        // ---- online softmax (base 2; the scale carries log2(e))
+        float mb = -INFINITY;
 #pragma unroll
-        for (int h = 0; h < GRP; ++h) bm[h] = sc[h];
-        block_reduce<GRP>(bm, sm.red, true);
-        float ps[GRP];
+        for (int i2 = 0; i2 < 16; ++i2) mb = fmaxf(mb, fmaxf(sc[i2].x, sc[i2].y));
+        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+        const float mnew = fmaxf(m_run, mb);
+        const float alpha = exp2f(m_run - mnew);
+        float ls = 0.f;
 #pragma unroll
-        for (int h = 0; h < GRP; ++h) {
-            const float p = t < ntail ? exp2f(sc[h] - bm[h]) : 0.f;
-            sm.pr[t][h] = p;
-            ps[h] = p;
+        for (int i2 = 0; i2 < 16; ++i2) {
+            sc[i2].x = exp2f(sc[i2].x - mnew);
+            sc[i2].y = exp2f(sc[i2].y - mnew);
+            ls += sc[i2].x + sc[i2].y;
         }
-        block_reduce<GRP>(ps, sm.red, false);
-#pragma unroll
-        for (int h = 0; h < GRP; ++h) { m_run[h] = bm[h]; l_run[h] = ps[h]; }
-        if (tid < D) {
-            for (int tt = 0; tt < ntail; ++tt) {
-                const float vv = In<Tin>::load1(vt + (size_t)tt * D + tid);
-#pragma unroll
-                for (int h = 0; h < GRP; ++h) acc[h] = fmaf(sm.pr[tt][h], vv, acc[h]);
+        l_run = fmaf(l_run, alpha, ls);
+        m_run = mnew;
+        __syncwarp();  // every lane is done with the K scales
+
+        // ---- V scales: rsV[g][t] = r^V_t s^V_{t,g}, rV[t], cV[d] * 2^18
+        {
+            const __half *sh = reinterpret_cast<const __half *>(vrec + R::kSOff);
+            const __half *rh = reinterpret_cast<const __half *>(vrec + R::kROff);
+            for (int idx = lane; idx < NG * kBlockTokens; idx += 32) {
+                const int t = idx / NG, g = idx % NG;
+                scr[g * kBlockTokens + t] = __half2float(sh[idx]) * __half2float(rh[t]);
             }
+            for (int t = lane; t < kBlockTokens; t += 32) scr[NG * kBlockTokens + t] = __half2float(rh[t]);
+            const __half *ch = reinterpret_cast<const __half *>(vrec + R::kCOff);
+            for (int d = lane; d < D; d += 32) scr[(NG + 1) * kBlockTokens + d] = __half2float(ch[d]) * kTwo18;
+        }
+        __syncwarp();
+        const float *rsV = scr, *rV = scr + NG * kBlockTokens, *cV = scr + (NG + 1) * kBlockTokens;
+
+        // ---- bias_{h,g} = sum_t p_t r_t m^V_{t,g} on the tensor cores
+        float accB[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+            const __half *mh = reinterpret_cast<const __half *>(vrec + R::kMOff);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const int T0 = 16 * ks + 2 * tig, T1 = T0 + 8;
+                uint32_t Ab[4] = {0u, 0u, 0u, 0u};
+                if (copy == 0) {
+                    split_hilo(sc[2 * ks].x * rV[T0], sc[2 * ks].y * rV[T0 + 1], Ab[0], Ab[1]);
+                    split_hilo(sc[2 * ks + 1].x * rV[T1], sc[2 * ks + 1].y * rV[T1 + 1], Ab[2], Ab[3]);
+                }
+                uint32_t bb0 = 0u, bb1 = 0u;
+                if (gl < NG) {
+                    __half2 p0 = __halves2half2(mh[T0 * NG + gl], mh[(T0 + 1) * NG + gl]);
+                    __half2 p1 = __halves2half2(mh[T1 * NG + gl], mh[(T1 + 1) * NG + gl]);
+                    bb0 = *reinterpret_cast<uint32_t *>(&p0);
+                    bb1 = *reinterpret_cast<uint32_t *>(&p1);
+                }
+                mma16816(accB, Ab, bb0, bb1);
+            }
+        }
+        const float2 bpair = f2(accB[0] + accB[2], accB[1] + accB[3]);  // (h, groups 2tig, 2tig+1)
+
+        // ---- P V, one group set at a time
+#pragma unroll
+        for (int i2 = 0; i2 < NNT; ++i2) orun[i2] = __fmul2_rn(orun[i2], f2(alpha, alpha));
+#pragma unroll
+        for (int st = 0; st < SETS; ++st) {
+            const int g = st * C + copy;
+            const bool gv = g < NG;
+            uint32_t Av[8][4];
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const int T0 = 16 * ks + 2 * tig, T1 = T0 + 8;
+                if (gv) {
+                    const float e = (ks >> 1) == 0 ? 64.f : (ks >> 1) == 1 ? 16.f : (ks >> 1) == 2 ? 4.f : 1.f;
+                    const float2 r0 = *reinterpret_cast<const float2 *>(rsV + g * kBlockTokens + T0);
+                    const float2 r1 = *reinterpret_cast<const float2 *>(rsV + g * kBlockTokens + T1);
+                    split_hilo(sc[2 * ks].x * r0.x * e, sc[2 * ks].y * r0.y * e, Av[ks][0], Av[ks][1]);
+                    split_hilo(sc[2 * ks + 1].x * r1.x * e, sc[2 * ks + 1].y * r1.y * e, Av[ks][2], Av[ks][3]);
+                } else {
+                    Av[ks][0] = Av[ks][1] = Av[ks][2] = Av[ks][3] = 0u;
+                }
+            }
+            // bias of (h, g) lives in lane 4*h + g/2 (copy 0)
+            const int gsrc = gv ? g : 0;
+            const float bx = __shfl_sync(0xffffffffu, bpair.x, 4 * h + gsrc / 2);
+            const float by = __shfl_sync(0xffffffffu, bpair.y, 4 * h + gsrc / 2);
+            const float bias = ((gsrc & 1) ? by : bx) * kTwoM18;
+#pragma unroll
+            for (int cc = 0; cc < C; ++cc) {
+                const int gg = st * C + cc;
+                if (gg >= NG) continue;
+#pragma unroll
+                for (int j4 = 0; j4 < kGroup / 8; ++j4) {
+                    const int nt = gg * (kGroup / 8) + j4;
+                    const uint2 vw2 = reinterpret_cast<const uint2 *>(vrec)[nt * 32 + lane];
+                    const uint32_t vw[2] = {vw2.x, vw2.y}, vw8[2] = {vw2.x >> 8, vw2.y >> 8};
+                    float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        uint32_t bb[2];
+#pragma unroll
+                        for (int cs = 0; cs < 2; ++cs) {
+                            const int m = 2 * ks + cs, am = m % 4;
+                            bb[cs] = code_pair(vw[am / 2], vw8[am / 2], 4 * (am % 2) + m / 4);
+                        }
+                        mma16816(acc4, Av[ks], bb[0], bb[1]);
+                    }
+                    if (cc == copy) {
+                        const float2 cv = *reinterpret_cast<const float2 *>(cV + 8 * nt + 2 * tig);
+                        const float2 o = f2(acc4[0] + acc4[2] + bias, acc4[1] + acc4[3] + bias);
+                        orun[nt] = __ffma2_rn(o, cv, orun[nt]);
+                    }
+                }
+            }
+        }
+
+        // ---- refill this stage with block b + 2
+        __syncwarp();
+        if (lane == 0 && b + 2 < b1)
+            issue_block(&sm.mbar[stage], sm.rec[stage][0], sm.rec[stage][1], kbase + (size_t)(b + 2) * R::kBytes,
+                        vbase + (size_t)(b + 2) * R::kBytes, R::kBytes);
+    }
+    if (failed_at >= 0) {
+        // let the copies this warp may still have in flight land (bounded), then report
+        if (lane == 0) {
+            for (int i = failed_at; i < failed_at + 2 && i < b1 - b0; ++i) mbar_wait(&sm.mbar[i & 1], (i >> 1) & 1);
+            status_or(a.status, KVARN_STATUS_TIMEOUT);
+        }
+        __syncwarp();
+        m_run = -INFINITY;
+        l_run = 0.f;
+#pragma unroll
+        for (int i2 = 0; i2 < NNT; ++i2) orun[i2] = f2(0.f, 0.f);
+    }
+
+    // ---- this warp's block partial: (m, l, o_rot) per head
+    const int slots = kMaxSplits + 1;
+    float *pbase = a.partials + (size_t)unit * slots * GRP * (D + 2);
+    {
+        float *pp = pbase + ((size_t)split * GRP + h) * (D + 2);
+        float lsum = l_run;
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+        if (copy == 0 && tig == 0) { pp[0] = m_run; pp[1] = lsum; }
+#pragma unroll
+        for (int nt = 0; nt < NNT; ++nt) {
+            if ((nt / (kGroup / 8)) % C == copy)
+                *reinterpret_cast<float2 *>(pp + 2 + 8 * nt + 2 * tig) = orun[nt];
         }
     }
 
-    // ---- write this split's partial (m, l, o) per head -------------------
-    float *part = a.partials + ((size_t)sh * (a.nsplit + 1) + split) * GRP * (D + 2);
+    // ---- residual tail (last split only): unrotated query, lanes over tokens
+    if (split == a.nsplit - 1) {
+        float *pt = pbase + (size_t)a.nsplit * GRP * (D + 2);  // tail slot
+        for (int i = lane; i < GRP * D; i += 32) (&sm.qbuf[0][0])[i] = In<Tin>::load1(qg + i) * a.scale_log2;
+        __syncwarp();
+        const Tin *kt = static_cast<const Tin *>(a.k_tail) + (size_t)unit * kBlockTokens * D;
+        const Tin *vt = static_cast<const Tin *>(a.v_tail) + (size_t)unit * kBlockTokens * D;
+        float st[4][GRP];
 #pragma unroll
-    for (int h = 0; h < GRP; ++h) {
-        if (tid < D) part[h * (D + 2) + 2 + tid] = acc[h];
-        if (tid == 0) { part[h * (D + 2)] = m_run[h]; part[h * (D + 2) + 1] = l_run[h]; }
+        for (int i = 0; i < 4; ++i) {
+            const int t = lane + 32 * i;
+#pragma unroll
+            for (int hh = 0; hh < GRP; ++hh) st[i][hh] = -INFINITY;
+            if (t < ntail) {
+#pragma unroll
+                for (int hh = 0; hh < GRP; ++hh) st[i][hh] = 0.f;
+                for (int d = 0; d < D; d += 8) {
+                    float kv[8];
+                    In<Tin>::load8(kt + (size_t)t * D + d, kv);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+#pragma unroll
+                        for (int hh = 0; hh < GRP; ++hh) st[i][hh] = fmaf(sm.qbuf[hh][d + e], kv[e], st[i][hh]);
+                }
+            }
+        }
+        float mt[GRP], lt[GRP];
+#pragma unroll
+        for (int hh = 0; hh < GRP; ++hh) {
+            float mx = fmaxf(fmaxf(st[0][hh], st[1][hh]), fmaxf(st[2][hh], st[3][hh]));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            mt[hh] = mx;
+            float ssum = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                st[i][hh] = (lane + 32 * i < ntail) ? exp2f(st[i][hh] - mx) : 0.f;
+                ssum += st[i][hh];
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
+            lt[hh] = ssum;
+        }
+        float ot[GRP][D / 32];
+#pragma unroll
+        for (int hh = 0; hh < GRP; ++hh)
+#pragma unroll
+            for (int c2 = 0; c2 < D / 32; ++c2) ot[hh][c2] = 0.f;
+        for (int t = 0; t < ntail; ++t) {
+            float pv[GRP];
+#pragma unroll
+            for (int hh = 0; hh < GRP; ++hh) {
+                const float v0 = st[0][hh], v1 = st[1][hh], v2 = st[2][hh], v3 = st[3][hh];
+                const float mine = (t >> 5) == 0 ? v0 : (t >> 5) == 1 ? v1 : (t >> 5) == 2 ? v2 : v3;
+                pv[hh] = __shfl_sync(0xffffffffu, mine, t & 31);
+            }
+#pragma unroll
+            for (int c2 = 0; c2 < D / 32; ++c2) {
+                const float vv = In<Tin>::load1(vt + (size_t)t * D + 32 * c2 + lane);
+#pragma unroll
+                for (int hh = 0; hh < GRP; ++hh) ot[hh][c2] = fmaf(pv[hh], vv, ot[hh][c2]);
+            }
+        }
+#pragma unroll
+        for (int hh = 0; hh < GRP; ++hh) {
+            float *pp = pt + (size_t)hh * (D + 2);
+            if (lane == 0) { pp[0] = ntail > 0 ? mt[hh] : -INFINITY; pp[1] = lt[hh]; }
+#pragma unroll
+            for (int c2 = 0; c2 < D / 32; ++c2) pp[2 + 32 * c2 + lane] = ot[hh][c2];
+        }
     }
+
+    // ---- arrival ticket; the last warp of this (sequence, kv head) combines
+    __syncwarp();
     __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        const unsigned prev = atomicAdd(a.tickets + sh, 1u);
-        sm.last = prev == (unsigned)a.nsplit;
-        if (sm.last) a.tickets[sh] = 0u;  // every CTA of this (s, kv head) has arrived
-    }
-    __syncthreads();
-    if (!sm.last) return;
+    unsigned prev = 0;
+    if (lane == 0) prev = atomicAdd(a.tickets + unit, 1u);
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    if (prev != (unsigned)a.nsplit - 1u) return;
+    if (lane == 0) a.tickets[unit] = 0u;
     __threadfence();
 
-    // ---- combine: log-sum-exp over splits, un-rotate, add the tail --------
-    const float *pbase = a.partials + (size_t)sh * (a.nsplit + 1) * GRP * (D + 2);
-    float *obuf = &sm.qp[0][0];   // [GRP][D] rotated part
-    float *otail = &sm.pw[0][0][0];  // [GRP][D] tail part (fits: T*NG*GRP >= GRP*D)
-    for (int idx = tid; idx < GRP * D; idx += kDecThreads) {
-        const int h = idx / D, d = idx % D;
+    float *obuf = reinterpret_cast<float *>(sm.rec[0][0]);   // [GRP][D] rotated part
+    float *otl = reinterpret_cast<float *>(sm.rec[1][0]);    // [GRP][D] tail part
+    for (int hh = 0; hh < GRP; ++hh) {
         float M = -INFINITY;
-        for (int i = 0; i <= a.nsplit; ++i) M = fmaxf(M, __ldcg(pbase + ((size_t)i * GRP + h) * (D + 2)));
-        float L = 0.f, orot = 0.f, otl = 0.f;
+        for (int i = 0; i <= a.nsplit; ++i) M = fmaxf(M, __ldcg(pbase + ((size_t)i * GRP + hh) * (D + 2)));
+        float L = 0.f;
+        float orot[D / 32], otail[D / 32];
+#pragma unroll
+        for (int c2 = 0; c2 < D / 32; ++c2) orot[c2] = otail[c2] = 0.f;
         if (M > -INFINITY) {
             for (int i = 0; i <= a.nsplit; ++i) {
-                const float *pp = pbase + ((size_t)i * GRP + h) * (D + 2);
+                const float *pp = pbase + ((size_t)i * GRP + hh) * (D + 2);
                 const float wgt = exp2f(__ldcg(pp) - M);
                 L = fmaf(__ldcg(pp + 1), wgt, L);
-                const float o = __ldcg(pp + 2 + d) * wgt;
-                if (i < a.nsplit) orot += o; else otl += o;
+#pragma unroll
+                for (int c2 = 0; c2 < D / 32; ++c2) {
+                    const float o = __ldcg(pp + 2 + 32 * c2 + lane) * wgt;
+                    if (i < a.nsplit) orot[c2] += o; else otail[c2] += o;
+                }
             }
         }
         const float inv = L > 0.f ? 1.f / L : 0.f;
-        obuf[idx] = orot * inv;
-        otail[idx] = otl * inv;
+#pragma unroll
+        for (int c2 = 0; c2 < D / 32; ++c2) {
+            obuf[hh * D + 32 * c2 + lane] = orot[c2] * inv;
+            otl[hh * D + 32 * c2 + lane] = otail[c2] * inv;
+        }
     }
-    __syncthreads();
-    smem_fwht(obuf, GRP, D, hb);
-    float *out = a.out + (size_t)sh * GRP * D;
-    for (int idx = tid; idx < GRP * D; idx += kDecThreads) out[idx] = obuf[idx] + otail[idx];
+    __syncwarp();
+    warp_fwht<D>(obuf, GRP, hb);
+    float *out = a.out + (size_t)unit * GRP * D;
+    for (int i = lane; i < GRP * D; i += 32) out[i] = obuf[i] + otl[i];
 }
 
 template <int D, int GRP, typename Tin>
-static cudaError_t launch_dec(const DecodeArgs &a, int hb, int S, int Hkv, cudaStream_t st)
+static cudaError_t launch_dec(const DecodeArgs &a, int hb, cudaStream_t st)
 {
-    const size_t smem = sizeof(DecSmem<D, GRP>);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, GRP, Tin>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    dim3 grid((unsigned)(S * Hkv), (unsigned)(a.nsplit + 1));
-    decode_kernel<D, GRP, Tin><<<grid, kDecThreads, smem, st>>>(a, hb);
+    const size_t smem = sizeof(DecWarpSmem<D, GRP>) * kDecWarps;
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, GRP, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const int items = a.num_units * a.nsplit;
+    dim3 grid((unsigned)((items + kDecWarps - 1) / kDecWarps));
+    decode_kernel<D, GRP, Tin><<<grid, kDecWarps * 32, smem, st>>>(a, hb);
     return cudaGetLastError();
 }
 
 template <int D, int GRP>
-static cudaError_t dispatch_dtype(int dtype, const DecodeArgs &a, int hb, int S, int Hkv, cudaStream_t st)
+static cudaError_t dispatch_dtype(int dtype, const DecodeArgs &a, int hb, cudaStream_t st)
 {
-    return dtype == KVARN_BF16 ? launch_dec<D, GRP, __nv_bfloat16>(a, hb, S, Hkv, st)
-                               : launch_dec<D, GRP, float>(a, hb, S, Hkv, st);
+    return dtype == KVARN_BF16 ? launch_dec<D, GRP, __nv_bfloat16>(a, hb, st) : launch_dec<D, GRP, float>(a, hb, st);
 }
 
 template <int D>
-static cudaError_t dispatch_grp(int dtype, const DecodeArgs &a, int hb, int S, int Hkv, cudaStream_t st)
+static cudaError_t dispatch_grp(int dtype, const DecodeArgs &a, int hb, cudaStream_t st)
 {
     switch (a.grp) {
-    case 1: return dispatch_dtype<D, 1>(dtype, a, hb, S, Hkv, st);
-    case 2: return dispatch_dtype<D, 2>(dtype, a, hb, S, Hkv, st);
-    case 4: return dispatch_dtype<D, 4>(dtype, a, hb, S, Hkv, st);
-    case 8: return dispatch_dtype<D, 8>(dtype, a, hb, S, Hkv, st);
+    case 1: return dispatch_dtype<D, 1>(dtype, a, hb, st);
+    case 2: return dispatch_dtype<D, 2>(dtype, a, hb, st);
+    case 4: return dispatch_dtype<D, 4>(dtype, a, hb, st);
+    case 8: return dispatch_dtype<D, 8>(dtype, a, hb, st);
     }
     return cudaErrorInvalidValue;
 }
@@ -369,11 +628,13 @@ static cudaError_t dispatch_grp(int dtype, const DecodeArgs &a, int hb, int S, i
 cudaError_t run_decode(const kvarn_config &c, const DecodeArgs &a, cudaStream_t st)
 {
     switch (c.head_dim) {
-    case 64: return dispatch_grp<64>(c.dtype, a, c.hadamard, c.num_seqs, c.num_kv_heads, st);
-    case 96: return dispatch_grp<96>(c.dtype, a, c.hadamard, c.num_seqs, c.num_kv_heads, st);
-    case 128: return dispatch_grp<128>(c.dtype, a, c.hadamard, c.num_seqs, c.num_kv_heads, st);
+    case 64: return dispatch_grp<64>(c.dtype, a, c.hadamard, st);
+    case 96: return dispatch_grp<96>(c.dtype, a, c.hadamard, st);
+    case 128: return dispatch_grp<128>(c.dtype, a, c.hadamard, st);
     }
     return cudaErrorInvalidValue;
 }
+
+int decode_warps_per_cta() { return kDecWarps; }
 
 }  // namespace kvarn

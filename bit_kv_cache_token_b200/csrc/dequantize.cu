@@ -25,17 +25,17 @@ dequantize_kernel(DequantArgs a)
                                ((size_t)sh * a.max_blocks + a.first_block + b) * R::kBytes;
     const int t = threadIdx.x;
     const float r = __half2float(*reinterpret_cast<const __half *>(rec + R::kROff + 2 * t));
+    const uint32_t *codes = reinterpret_cast<const uint32_t *>(rec);
     float x[D];
 #pragma unroll
     for (int g = 0; g < D / kGroup; ++g) {
-        const __half2 sm = *reinterpret_cast<const __half2 *>(rec + R::kGpOff + (t * (D / kGroup) + g) * 4);
-        const float s = __low2float(sm), m = __high2float(sm);
-        const uint2 cw = *reinterpret_cast<const uint2 *>(rec + t * (D / 4) + 8 * g);
+        const float s = __half2float(reinterpret_cast<const __half *>(rec + R::kSOff)[t * (D / kGroup) + g]);
+        const float m = __half2float(reinterpret_cast<const __half *>(rec + R::kMOff)[t * (D / kGroup) + g]);
 #pragma unroll
         for (int i = 0; i < kGroup; ++i) {
-            const uint32_t word = i < 16 ? cw.x : cw.y;
-            const float code = (float)((word >> (2 * (i & 15))) & 3u);
             const int d = g * kGroup + i;
+            const int bit = tensor ? v_code_bit(t, d) : k_code_bit<D>(t, d);
+            const float code = (float)((codes[bit >> 5] >> (bit & 31)) & 3u);
             const float c = __half2float(*reinterpret_cast<const __half *>(rec + R::kCOff + 2 * d));
             x[d] = r * c * fmaf(s, code, m);
         }

@@ -159,11 +159,13 @@ int kvarn_decode_attention(const kvarn_config *cfg, const void *q, int num_q_hea
     const size_t need = kvarn_decode_workspace_bytes(cfg, num_q_heads);
     if (!workspace || !aligned16(workspace) || workspace_bytes < need) return KVARN_EWORKSPACE;
 
+    // one warp per (sequence, kv head, split); splits sized so that all warps
+    // are resident at once (one CTA of decode_warps_per_cta() warps per SM)
     const int units = cfg->num_seqs * cfg->num_kv_heads;
     const int nblk = max_tokens / cfg->block_tokens;
-    int nsplit = 0, bps = 1;
+    int nsplit = 1, bps = nblk > 0 ? nblk : 1;
     if (nblk > 0) {
-        int ns = (2 * num_sms() + units - 1) / units;
+        int ns = num_sms() * decode_warps_per_cta() / units;
         ns = ns < 1 ? 1 : ns;
         ns = ns > nblk ? nblk : ns;
         ns = ns > kMaxSplits ? kMaxSplits : ns;
@@ -181,7 +183,7 @@ int kvarn_decode_attention(const kvarn_config *cfg, const void *q, int num_q_hea
     const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)cfg->head_dim);
     a.scale_log2 = scale * 1.4426950408889634f;
     a.num_kv_heads = cfg->num_kv_heads; a.grp = grp; a.max_blocks = cfg->max_blocks;
-    a.max_tokens = max_tokens; a.nsplit = nsplit; a.blocks_per_split = bps;
+    a.max_tokens = max_tokens; a.num_units = units; a.nsplit = nsplit; a.blocks_per_split = bps;
     return cuda_status(run_decode(*cfg, a, static_cast<cudaStream_t>(stream)));
 }
 

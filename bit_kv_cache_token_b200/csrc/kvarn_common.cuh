@@ -16,18 +16,41 @@ namespace kvarn {
 constexpr int kBlockTokens = 128;
 constexpr int kGroup = 32;
 
-// Byte layout of one block record (see kvarn.h): codes, (s, m) pairs,
-// token scales r, channel scales c, padded to 128 bytes.
+// Byte layout of one block record (see kvarn.h): 2-bit codes in the K or V
+// fragment order, binary16 steps s[t][g], minima m[t][g], token scales r,
+// channel scales c, padded to 128 bytes.
 template <int D>
 struct Record {
     static constexpr int kCodes = kBlockTokens * D / 4;
     static constexpr int kGroups = D / kGroup;
-    static constexpr int kGpOff = kCodes;
-    static constexpr int kROff = kGpOff + kBlockTokens * kGroups * 4;
+    static constexpr int kSOff = kCodes;
+    static constexpr int kMOff = kSOff + kBlockTokens * kGroups * 2;
+    static constexpr int kROff = kMOff + kBlockTokens * kGroups * 2;
     static constexpr int kCOff = kROff + 2 * kBlockTokens;
     static constexpr int kRaw = kCOff + 2 * D;
     static constexpr int kBytes = (kRaw + 127) / 128 * 128;
 };
+
+// Bit index, inside the code area, of the code of (token t, channel k) of a
+// K record (fragment order of kvarn.h).
+template <int D>
+__host__ __device__ constexpr int k_code_bit(int t, int k)
+{
+    constexpr int F = D / 64;
+    const int u = t / 16, n = (t % 16) / 8, lane = 4 * (t % 8) + (k % 8) / 2, half = k % 2, q = k / 8;
+    int word, pos;
+    if (q < 8 * F) { word = n * F + q / 8; pos = q % 8; }
+    else { word = 2 * F; pos = q - 8 * F + 4 * n; }
+    return ((u * 32 + lane) * (D / 32) + word) * 32 + 16 * half + 2 * pos;
+}
+
+// Same for a V record (token t, channel d).
+__host__ __device__ constexpr int v_code_bit(int t, int d)
+{
+    const int j = d / 8, lane = 4 * (d % 8) + (t % 8) / 2, half = t % 2, a = (t % 32) / 8;
+    const int word = a / 2, pos = 4 * (a % 2) + t / 32;
+    return ((j * 32 + lane) * 2 + word) * 32 + 16 * half + 2 * pos;
+}
 
 __host__ __device__ inline size_t record_bytes_rt(int D)
 {

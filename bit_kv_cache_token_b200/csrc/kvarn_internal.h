@@ -46,7 +46,8 @@ struct DecodeArgs {
     uint32_t *tickets;          // [S*Hkv]
     float scale_log2;           // softmax scale * log2(e)
     int num_kv_heads, grp, max_blocks, max_tokens;
-    int nsplit, blocks_per_split;
+    int num_units;              // S * Hkv
+    int nsplit, blocks_per_split;  // warps per unit, blocks per warp
 };
 
 cudaError_t run_quantize(const kvarn_config &c, const QuantArgs &a, cudaStream_t st);
@@ -57,5 +58,8 @@ cudaError_t run_set_length(int32_t *n_tokens, int num_seqs, int value, cudaStrea
 
 // Largest split count the decode workspace is sized for.
 constexpr int kMaxSplits = 64;
+
+// Warps per decode CTA (one CTA per SM by shared memory).
+int decode_warps_per_cta();
 
 }  // namespace kvarn

@@ -81,10 +81,10 @@ __device__ __forceinline__ void load_block(const Tin *rows, float2 (&X)[4][16])
 }
 
 // Quantise the block held in X (destroyed) into rec_out (global, 16-byte
-// aligned, Record<D>::kBytes).  dbg: NULL or fp32 [T + D + 2*T*D/32] unrounded
+// aligned, Record<D>::kBytes); tensor 0 = K code order, 1 = V code order.  dbg: NULL or fp32 [T + D + 2*T*D/32] unrounded
 // r, c, s, m.  All D threads of the CTA must call this.
 template <int D, int HB>
-__device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
+__device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps, int tensor,
                                unsigned char *__restrict__ rec_out, float *__restrict__ dbg,
                                int32_t *status)
 {
@@ -213,7 +213,12 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
     __syncthreads();  // every warp is done with the shared transposes
 
     // ---- 3. 2-bit asymmetric round-to-nearest per (token, group) ----------
+    // Codes go to the record in the fragment order the decode kernel reads
+    // (see kvarn.h).  K: the 4 codes of channels 8x + 2*tig + half (x = 0..3)
+    // of one token fill one byte.  V: the codes of one channel for this
+    // thread's 4 tokens (l + 32r) fill one byte.
     unsigned char *rec = sm.u.rec;
+    uint32_t vbytes[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // V: channel i in byte i%4 of vbytes[i/4]
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         const int t = l + 32 * r;
@@ -233,22 +238,30 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
         // 12582912 = 1.5 * 2^23: adding it rounds the level to an integer
         // (ties to even) and leaves that integer in the low mantissa bits.
         const float2 magic = f2(12582912.f, 12582912.f);
-        uint32_t words[2] = {0u, 0u};
+        uint32_t kbytes[4] = {0u, 0u, 0u, 0u};  // K: byte (tig, half) at bits 8*half of kbytes[tig]
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
             const float2 lev = __fadd2_rn(__ffma2_rn(z[k], kq2, nmk), magic);
             const uint32_t c0 = __float_as_uint(lev.x) & 3u, c1 = __float_as_uint(lev.y) & 3u;
-            const int sh = (4 * k) & 31;  // channel 2k sits at bit 2*(2k) of its word
-            words[k >> 3] |= (c0 << sh) | (c1 << (sh + 2));
+            // local channels 2k (c0) and 2k+1 (c1): x = k/4, tig = k%4
+            kbytes[k & 3] |= (c0 << (2 * (k >> 2))) | (c1 << (8 + 2 * (k >> 2)));
+            vbytes[k >> 1] |= (c0 << (16 * (k & 1) + 2 * r)) | (c1 << (16 * (k & 1) + 8 + 2 * r));
         }
-        *reinterpret_cast<uint2 *>(rec + t * (D / 4) + 8 * j) = make_uint2(words[0], words[1]);
+        if (tensor == 0) {
+#pragma unroll
+            for (int tig = 0; tig < 4; ++tig) {
+                const int kch = 32 * j + 2 * tig;  // channel with x = 0, half = 0
+                rec[k_code_bit<D>(t, kch) / 8] = (unsigned char)(kbytes[tig] & 0xFFu);
+                rec[k_code_bit<D>(t, kch + 1) / 8] = (unsigned char)(kbytes[tig] >> 8);
+            }
+        }
         const float s = range * w[r] * (1.f / 3.f);
         const float m = mn * w[r];
         const __half hs = __float2half_rn(s), hm = __float2half_rn(m);
         if (__hisinf(hs) || __hisnan(hs) || __hisinf(hm) || __hisnan(hm))
             status_or(status, KVARN_STATUS_NONFINITE);
-        __half2 sm2 = __halves2half2(hs, hm);
-        *reinterpret_cast<__half2 *>(rec + R::kGpOff + (t * (D / 32) + j) * 4) = sm2;
+        reinterpret_cast<__half *>(rec + R::kSOff)[t * (D / 32) + j] = hs;
+        reinterpret_cast<__half *>(rec + R::kMOff)[t * (D / 32) + j] = hm;
         if (j == 0) {
             const __half hr = __float2half_rn(rt[r]);
             if (__hisinf(hr) || __hisnan(hr)) status_or(status, KVARN_STATUS_NONFINITE);
@@ -259,6 +272,11 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
             dbg[kBlockTokens + D + t * (D / 32) + j] = s;
             dbg[kBlockTokens + D + kBlockTokens * (D / 32) + t * (D / 32) + j] = m;
         }
+    }
+    if (tensor == 1) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            rec[v_code_bit(l, 32 * j + i) / 8] = (unsigned char)(vbytes[i >> 2] >> (8 * (i & 3)));
     }
     {
         const __half hc = __float2half_rn(cd);

@@ -59,6 +59,8 @@ extern "C" {
 #define KVARN_STATUS_CAPACITY  1  /* append needed block >= max_blocks     */
 #define KVARN_STATUS_NONFINITE 2  /* a scale rounded to inf/nan in binary16 */
 #define KVARN_STATUS_LENGTH    4  /* n_tokens[s] > max_tokens at decode     */
+#define KVARN_STATUS_TIMEOUT   8  /* a staged copy did not arrive in time;  */
+                                  /* the affected partial result is dropped */
 
 typedef enum { KVARN_F32 = 0, KVARN_BF16 = 1 } kvarn_dtype;
 
@@ -92,14 +94,25 @@ typedef struct {
  *
  * k_records, v_records: [num_seqs][num_kv_heads][max_blocks] block records of
  *   kvarn_record_bytes(cfg) bytes each.  A record holds, for one block of
- *   T = block_tokens tokens and D channels:
- *     codes    T*D/4 bytes; channel d of token t is byte t*D/4 + d/4,
- *              bits 2*(d%4)..2*(d%4)+1 (code 0..3)
- *     gparams  T*(D/group) pairs of binary16 (step s, minimum m), step first
+ *   T = block_tokens tokens and D channels (G = D/group groups):
+ *     codes    T*D/4 bytes of 2-bit codes (0..3), in the fragment order below
+ *     s        T*G binary16 steps, token-major: s[t*G + g]
+ *     m        T*G binary16 minima, token-major: m[t*G + g]
  *     r        T binary16 token scales
  *     c        D binary16 channel scales
  *     zero padding to a multiple of 128 bytes.
  *   The dequantised, still rotated value is r_t * c_d * (s * code + m).
+ *   Code order.  Every code sits in a 32-bit little-endian word at bit
+ *   16*half + 2*pos, 0 <= pos < 8, so that one AND of a word with
+ *   0x00030003 << 2*(pos % 4) (after a shift by 8 when pos >= 4) yields two
+ *   codes as the two halves of an exact binary16 pair.
+ *   K record (token t, channel k):  u = t/16, l = 4*(t%8) + (k%8)/2,
+ *     half = k%2, q = k/8, n = (t%16)/8, F = D/64;
+ *     q < 8F:  word = n*F + q/8, pos = q%8;  else (D = 96): word = 2F,
+ *     pos = q - 8F + 4n;  byte offset of the word = ((u*32 + l)*(D/32) + word)*4.
+ *   V record (token t, channel d):  j = d/8, l = 4*(d%8) + (t%8)/2,
+ *     half = t%2, a = (t%32)/8, word = a/2, pos = 4*(a%2) + t/32;
+ *     byte offset of the word = ((j*32 + l)*2 + word)*4.
  * k_tail, v_tail: [num_seqs][num_kv_heads][block_tokens][D] in cfg->dtype;
  *   tokens n - n % T .. n - 1 of each sequence, unrotated, as given.
  * n_tokens: [num_seqs] int32, tokens held per sequence (blocks then tail).

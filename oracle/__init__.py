@@ -54,14 +54,17 @@ def lib():
         L.kvo_f16_value.restype = ctypes.c_double
         L.kvo_record_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
         L.kvo_record_bytes.restype = ctypes.c_size_t
-        L.kvo_pack_record.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _u8p, _dp, _dp, _dp, _dp, _u8p]
-        L.kvo_unpack_record.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _u8p, _u8p, _dp, _dp, _dp, _dp]
-        L.kvo_dequantize_record.argtypes = [_u8p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        L.kvo_pack_record.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _u8p, _dp, _dp, _dp,
+                                      _dp, _u8p]
+        L.kvo_unpack_record.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _u8p, _u8p, _dp, _dp,
+                                        _dp, _dp]
+        L.kvo_dequantize_record.argtypes = [_u8p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                             ctypes.c_int, _dp]
         L.kvo_attention.argtypes = [_dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp,
                                     ctypes.c_double, _dp]
         L.kvo_quantize_many.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
-                                        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int]
+                                        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                        ctypes.c_int]
         L.kvo_quantize_many.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -128,31 +131,37 @@ def f16_value(bits: int) -> float:
 
 
 # ------------------------------------------------------------------ records
+# Code layouts of a record: NATURAL (token-major, any T), K_ORDER / V_ORDER (the
+# fragment orders the library writes for K and V blocks of 128 tokens).
+NATURAL, K_ORDER, V_ORDER = 0, 1, 2
+
+
 def record_bytes(T: int, D: int, group: int = 32) -> int:
     return int(lib().kvo_record_bytes(T, D, group))
 
 
-def pack_record(q: dict, group: int = 32) -> np.ndarray:
+def pack_record(q: dict, layout: int = NATURAL, group: int = 32) -> np.ndarray:
     codes = np.ascontiguousarray(q["codes"], dtype=np.uint8)
     T, D = codes.shape
     rec = np.empty(record_bytes(T, D, group), dtype=np.uint8)
-    lib().kvo_pack_record(T, D, group, codes, _f64(q["r"]), _f64(q["c"]), _f64(q["s"]), _f64(q["m"]), rec)
+    lib().kvo_pack_record(T, D, group, layout, codes, _f64(q["r"]), _f64(q["c"]), _f64(q["s"]), _f64(q["m"]), rec)
     return rec
 
 
-def unpack_record(rec, T: int, D: int, group: int = 32) -> dict:
+def unpack_record(rec, T: int, D: int, layout: int = NATURAL, group: int = 32) -> dict:
     rec = np.ascontiguousarray(rec, dtype=np.uint8)
     ng = D // group
     out = dict(codes=np.empty((T, D), dtype=np.uint8), r=np.empty(T), c=np.empty(D), s=np.empty((T, ng)),
                m=np.empty((T, ng)))
-    lib().kvo_unpack_record(T, D, group, rec, out["codes"], out["r"], out["c"], out["s"], out["m"])
+    lib().kvo_unpack_record(T, D, group, layout, rec, out["codes"], out["r"], out["c"], out["s"], out["m"])
     return out
 
 
-def dequantize_record(rec, T: int, D: int, hb: int, rotated: bool = False, group: int = 32) -> np.ndarray:
+def dequantize_record(rec, T: int, D: int, hb: int, rotated: bool = False, layout: int = NATURAL,
+                      group: int = 32) -> np.ndarray:
     rec = np.ascontiguousarray(rec, dtype=np.uint8)
     out = np.empty((T, D), dtype=np.float64)
-    lib().kvo_dequantize_record(rec, T, D, group, hb, 1 if rotated else 0, out)
+    lib().kvo_dequantize_record(rec, T, D, group, layout, hb, 1 if rotated else 0, out)
     return out
 
 
@@ -170,13 +179,16 @@ def attention(q, K, V, scale: float) -> np.ndarray:
 
 
 def decode_from_cache(q, k_records, v_records, k_tail, v_tail, n_tokens: int, T: int, hb: int,
-                      scale: float, group: int = 32) -> np.ndarray:
+                      scale: float, group: int = 32, layouts=None) -> np.ndarray:
     """Decode attention for one sequence from packed records plus the residual tail.
 
     q (Hq, D); k_records/v_records (Hkv, nblk_capacity, record_bytes) uint8; k_tail/v_tail (Hkv, T, D) values
     as stored (any float dtype, widened exactly).  The first n_tokens // T blocks are dequantised to the
-    original basis, followed by n_tokens % T tail tokens; then explicit softmax attention.
+    original basis, followed by n_tokens % T tail tokens; then explicit softmax attention.  layouts =
+    (K layout, V layout); by default the library's K_ORDER / V_ORDER for T = 128, NATURAL otherwise.
     """
+    if layouts is None:
+        layouts = (K_ORDER, V_ORDER) if T == 128 else (NATURAL, NATURAL)
     q = _f64(q)
     Hq, D = q.shape
     Hkv = k_records.shape[0]
@@ -185,8 +197,8 @@ def decode_from_cache(q, k_records, v_records, k_tail, v_tail, n_tokens: int, T:
     V = np.empty((Hkv, n_tokens, D))
     for h in range(Hkv):
         for b in range(nblk):
-            K[h, b * T:(b + 1) * T] = dequantize_record(k_records[h, b], T, D, hb, False, group)
-            V[h, b * T:(b + 1) * T] = dequantize_record(v_records[h, b], T, D, hb, False, group)
+            K[h, b * T:(b + 1) * T] = dequantize_record(k_records[h, b], T, D, hb, False, layouts[0], group)
+            V[h, b * T:(b + 1) * T] = dequantize_record(v_records[h, b], T, D, hb, False, layouts[1], group)
         K[h, nblk * T:] = np.asarray(k_tail[h, :ntail], dtype=np.float64)
         V[h, nblk * T:] = np.asarray(v_tail[h, :ntail], dtype=np.float64)
     return attention(q, K, V, scale)
@@ -194,7 +206,7 @@ def decode_from_cache(q, k_records, v_records, k_tail, v_tail, n_tokens: int, T:
 
 # ------------------------------------------------------------ bulk, threads
 def quantize_many(x: np.ndarray, dtype: str, T: int, D: int, hb: int, sweeps: int = 4, group: int = 32,
-                  nthreads: int = 1):
+                  nthreads: int = 1, layout: int = NATURAL):
     """Quantise consecutive T x D blocks of a raw fp32 / bf16 (as uint16) array on nthreads threads.
 
     Returns (records uint8 [nunits, record_bytes], threads used).
@@ -204,6 +216,6 @@ def quantize_many(x: np.ndarray, dtype: str, T: int, D: int, hb: int, sweeps: in
     nunits = x.size // (T * D)
     rb = record_bytes(T, D, group)
     recs = np.empty((nunits, rb), dtype=np.uint8)
-    used = lib().kvo_quantize_many(x.ctypes.data, code, nunits, T, D, hb, sweeps, group, recs.ctypes.data,
-                                   nthreads)
+    used = lib().kvo_quantize_many(x.ctypes.data, code, nunits, T, D, hb, sweeps, group, layout,
+                                   recs.ctypes.data, nthreads)
     return recs, used

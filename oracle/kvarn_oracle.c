@@ -223,12 +223,23 @@ double kvo_f16_value(uint16_t h)
 
 /*
  * One record per (sequence, kv head, block) and per tensor (K or V):
- *   codes    T x D/4 bytes, token-major; channel d of token t sits in byte
- *            t*D/4 + d/4 at bits 2*(d%4) .. 2*(d%4)+1
- *   gparams  T x D/G pairs (binary16 step s, binary16 min m), s first
+ *   codes    T*D/4 bytes of 2-bit codes
+ *   s        T*(D/G) binary16 steps, token-major  s[t*(D/G) + g]
+ *   m        T*(D/G) binary16 minima, token-major m[t*(D/G) + g]
  *   r        T binary16 token scales
  *   c        D binary16 channel scales
  * and zero padding up to a multiple of 128 bytes.
+ *
+ * Where the codes sit (layout):
+ *   0 natural  byte t*D/4 + d/4, bits 2*(d%4)   (any T; oracle-only tests)
+ *   1 K order  (T = 128) word w of lane l of 16-token unit u, bit 16*half+2*pos:
+ *              u = t/16, l = 4*(t%8) + (d%8)/2, half = d%2, q = d/8, n = (t%16)/8,
+ *              F = D/64; q < 8F: w = n*F + q/8, pos = q%8; else w = 2F, pos = q-8F+4n;
+ *              word at byte ((u*32 + l)*(D/32) + w)*4
+ *   2 V order  (T = 128) j = d/8, l = 4*(d%8) + (t%8)/2, half = t%2, a = (t%32)/8,
+ *              w = a/2, pos = 4*(a%2) + t/32; word at byte ((j*32 + l)*2 + w)*4,
+ *              bit 16*half+2*pos
+ * The library writes K blocks in layout 1 and V blocks in layout 2.
  */
 size_t kvo_record_bytes(int T, int D, int G)
 {
@@ -236,26 +247,57 @@ size_t kvo_record_bytes(int T, int D, int G)
     return (b + 127) / 128 * 128;
 }
 
-void kvo_pack_record(int T, int D, int G, const uint8_t *codes, const double *r,
+/* Byte offset and bit (within that byte) of the code of (token t, channel d). */
+static void kvo_code_site(int T, int D, int layout, int t, int d, size_t *byte, int *bit)
+{
+    if (layout == 0) {
+        *byte = (size_t)t * D / 4 + d / 4;
+        *bit = 2 * (d % 4);
+        return;
+    }
+    size_t word;
+    int wbit;
+    if (layout == 1) {
+        const int u = t / 16, l = 4 * (t % 8) + (d % 8) / 2, half = d % 2, q = d / 8, n = (t % 16) / 8;
+        const int F = D / 64;
+        int w, pos;
+        if (q < 8 * F) { w = n * F + q / 8; pos = q % 8; }
+        else { w = 2 * F; pos = q - 8 * F + 4 * n; }
+        word = ((size_t)(u * 32 + l) * (D / 32) + w) * 4;
+        wbit = 16 * half + 2 * pos;
+    } else {
+        const int j = d / 8, l = 4 * (d % 8) + (t % 8) / 2, half = t % 2, a = (t % 32) / 8;
+        const int w = a / 2, pos = 4 * (a % 2) + t / 32;
+        word = ((size_t)(j * 32 + l) * 2 + w) * 4;
+        wbit = 16 * half + 2 * pos;
+    }
+    (void)T;
+    *byte = word + wbit / 8;
+    *bit = wbit % 8;
+}
+
+void kvo_pack_record(int T, int D, int G, int layout, const uint8_t *codes, const double *r,
                      const double *c, const double *s, const double *m, uint8_t *rec)
 {
     const int ng = D / G;
     memset(rec, 0, kvo_record_bytes(T, D, G));
     uint8_t *pc = rec;
-    uint8_t *pg = pc + (size_t)T * D / 4;
-    uint8_t *pr = pg + (size_t)T * ng * 4;
+    uint8_t *ps = pc + (size_t)T * D / 4;
+    uint8_t *pm = ps + (size_t)T * ng * 2;
+    uint8_t *pr = pm + (size_t)T * ng * 2;
     uint8_t *pcs = pr + 2 * (size_t)T;
     for (int t = 0; t < T; ++t)
-        for (int d = 0; d < D; ++d)
-            pc[(size_t)t * D / 4 + d / 4] |= (uint8_t)((codes[(size_t)t * D + d] & 3) << (2 * (d % 4)));
-    for (int t = 0; t < T; ++t)
-        for (int g = 0; g < ng; ++g) {
-            uint16_t hs = kvo_f16_bits(s[(size_t)t * ng + g]);
-            uint16_t hm = kvo_f16_bits(m[(size_t)t * ng + g]);
-            uint8_t *p = pg + ((size_t)t * ng + g) * 4;
-            p[0] = (uint8_t)(hs & 0xFF); p[1] = (uint8_t)(hs >> 8);
-            p[2] = (uint8_t)(hm & 0xFF); p[3] = (uint8_t)(hm >> 8);
+        for (int d = 0; d < D; ++d) {
+            size_t byte;
+            int bit;
+            kvo_code_site(T, D, layout, t, d, &byte, &bit);
+            pc[byte] |= (uint8_t)((codes[(size_t)t * D + d] & 3) << bit);
         }
+    for (size_t i = 0; i < (size_t)T * ng; ++i) {
+        uint16_t hs = kvo_f16_bits(s[i]), hm = kvo_f16_bits(m[i]);
+        ps[2 * i] = (uint8_t)(hs & 0xFF); ps[2 * i + 1] = (uint8_t)(hs >> 8);
+        pm[2 * i] = (uint8_t)(hm & 0xFF); pm[2 * i + 1] = (uint8_t)(hm >> 8);
+    }
     for (int t = 0; t < T; ++t) {
         uint16_t h = kvo_f16_bits(r[t]);
         pr[2 * t] = (uint8_t)(h & 0xFF); pr[2 * t + 1] = (uint8_t)(h >> 8);
@@ -275,22 +317,26 @@ static double kvo_load_f16(const uint8_t *p)
  * Read a record back: codes (T x D, one per byte) and the stored scales,
  * widened exactly from binary16.
  */
-void kvo_unpack_record(int T, int D, int G, const uint8_t *rec, uint8_t *codes,
+void kvo_unpack_record(int T, int D, int G, int layout, const uint8_t *rec, uint8_t *codes,
                        double *r, double *c, double *s, double *m)
 {
     const int ng = D / G;
     const uint8_t *pc = rec;
-    const uint8_t *pg = pc + (size_t)T * D / 4;
-    const uint8_t *pr = pg + (size_t)T * ng * 4;
+    const uint8_t *ps = pc + (size_t)T * D / 4;
+    const uint8_t *pm = ps + (size_t)T * ng * 2;
+    const uint8_t *pr = pm + (size_t)T * ng * 2;
     const uint8_t *pcs = pr + 2 * (size_t)T;
     for (int t = 0; t < T; ++t)
-        for (int d = 0; d < D; ++d)
-            codes[(size_t)t * D + d] = (uint8_t)((pc[(size_t)t * D / 4 + d / 4] >> (2 * (d % 4))) & 3);
-    for (int t = 0; t < T; ++t)
-        for (int g = 0; g < ng; ++g) {
-            s[(size_t)t * ng + g] = kvo_load_f16(pg + ((size_t)t * ng + g) * 4);
-            m[(size_t)t * ng + g] = kvo_load_f16(pg + ((size_t)t * ng + g) * 4 + 2);
+        for (int d = 0; d < D; ++d) {
+            size_t byte;
+            int bit;
+            kvo_code_site(T, D, layout, t, d, &byte, &bit);
+            codes[(size_t)t * D + d] = (uint8_t)((pc[byte] >> bit) & 3);
         }
+    for (size_t i = 0; i < (size_t)T * ng; ++i) {
+        s[i] = kvo_load_f16(ps + 2 * i);
+        m[i] = kvo_load_f16(pm + 2 * i);
+    }
     for (int t = 0; t < T; ++t) r[t] = kvo_load_f16(pr + 2 * t);
     for (int d = 0; d < D; ++d) c[d] = kvo_load_f16(pcs + 2 * d);
 }
@@ -300,7 +346,7 @@ void kvo_unpack_record(int T, int D, int G, const uint8_t *rec, uint8_t *codes,
  *   Xhat_rot[t][d] = r_t * c_d * (s_{t,g} * code + m_{t,g})
  * and, unless rotated != 0, rotate back to the original channel basis.
  */
-void kvo_dequantize_record(const uint8_t *rec, int T, int D, int G, int hb, int rotated,
+void kvo_dequantize_record(const uint8_t *rec, int T, int D, int G, int layout, int hb, int rotated,
                            double *Xhat)
 {
     const int ng = D / G;
@@ -310,7 +356,7 @@ void kvo_dequantize_record(const uint8_t *rec, int T, int D, int G, int hb, int 
     double *s = (double *)malloc(sizeof(double) * (size_t)T * ng);
     double *m = (double *)malloc(sizeof(double) * (size_t)T * ng);
     double *row = (double *)malloc(sizeof(double) * (size_t)D);
-    kvo_unpack_record(T, D, G, rec, codes, r, c, s, m);
+    kvo_unpack_record(T, D, G, layout, rec, codes, r, c, s, m);
     for (int t = 0; t < T; ++t) {
         for (int d = 0; d < D; ++d) {
             const int g = d / G;
@@ -377,7 +423,7 @@ static double kvo_load_input(const void *x, int dtype, size_t i)
 }
 
 typedef struct {
-    const void *x; int dtype; int64_t nunits; int T, D, hb, sweeps, G;
+    const void *x; int dtype; int64_t nunits; int T, D, hb, sweeps, G, layout;
     uint8_t *records; int nthreads, tid;
 } kvo_job;
 
@@ -395,7 +441,7 @@ static void *kvo_worker(void *arg)
     for (int64_t u = j->tid; u < j->nunits; u += j->nthreads) {
         for (size_t i = 0; i < n; ++i) X[i] = kvo_load_input(j->x, j->dtype, (size_t)u * n + i);
         kvo_quantize_block(X, j->T, j->D, j->hb, j->sweeps, j->G, NULL, r, c, s, m, NULL, codes);
-        kvo_pack_record(j->T, j->D, j->G, codes, r, c, s, m, j->records + (size_t)u * rb);
+        kvo_pack_record(j->T, j->D, j->G, j->layout, codes, r, c, s, m, j->records + (size_t)u * rb);
     }
     free(codes); free(m); free(s); free(c); free(r); free(X);
     return NULL;
@@ -403,17 +449,17 @@ static void *kvo_worker(void *arg)
 
 /*
  * Quantise nunits consecutive T x D input blocks (fp32 or bf16) into packed
- * records, on nthreads POSIX threads.  Returns the number of threads used.
+ * records with code layout `layout`, on nthreads POSIX threads.  Returns the number of threads used.
  */
 int kvo_quantize_many(const void *x, int dtype, int64_t nunits, int T, int D, int hb,
-                      int sweeps, int G, uint8_t *records, int nthreads)
+                      int sweeps, int G, int layout, uint8_t *records, int nthreads)
 {
     if (nthreads < 1) nthreads = 1;
     if (nthreads > 256) nthreads = 256;
     pthread_t th[256];
     kvo_job jobs[256];
     for (int i = 0; i < nthreads; ++i) {
-        jobs[i] = (kvo_job){x, dtype, nunits, T, D, hb, sweeps, G, records, nthreads, i};
+        jobs[i] = (kvo_job){x, dtype, nunits, T, D, hb, sweeps, G, layout, records, nthreads, i};
         pthread_create(&th[i], NULL, kvo_worker, &jobs[i]);
     }
     for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);

@@ -21,18 +21,37 @@ SCALE_RTOL = 1e-5
 DECODE_ATOL = 2e-3
 
 
-def view_record(rec, T: int, D: int, G: int = 32) -> dict:
+def code_bit_index(T: int, D: int, layout: int) -> np.ndarray:
+    """Bit index of each (token, channel) code inside the code area, from the record format in kvarn.h."""
+    t = np.arange(T)[:, None]
+    d = np.arange(D)[None, :]
+    if layout == oracle.NATURAL:
+        return (t * D // 4 + d // 4) * 8 + 2 * (d % 4)
+    if layout == oracle.K_ORDER:
+        F = D // 64
+        u, n, lane, half, q = t // 16, (t % 16) // 8, 4 * (t % 8) + (d % 8) // 2, d % 2, d // 8
+        word = np.where(q < 8 * F, n * F + q // 8, 2 * F)
+        pos = np.where(q < 8 * F, q % 8, q - 8 * F + 4 * n)
+        return ((u * 32 + lane) * (D // 32) + word) * 32 + 16 * half + 2 * pos
+    j, lane, half, a = d // 8, 4 * (d % 8) + (t % 8) // 2, t % 2, (t % 32) // 8
+    word, pos = a // 2, 4 * (a % 2) + t // 32
+    return ((j * 32 + lane) * 2 + word) * 32 + 16 * half + 2 * pos
+
+
+def view_record(rec, T: int, D: int, layout: int, G: int = 32) -> dict:
     rec = np.ascontiguousarray(np.asarray(rec, dtype=np.uint8))
     nc, ng = T * D // 4, D // G
-    cb = rec[:nc].reshape(T, D // 4)
-    codes = np.stack([(cb >> (2 * i)) & 3 for i in range(4)], axis=-1).reshape(T, D)
-    gp = rec[nc:nc + T * ng * 4].view(np.float16).reshape(T, ng, 2)
-    ro = nc + T * ng * 4
+    bits = code_bit_index(T, D, layout)
+    codes = (rec[bits // 8] >> (bits % 8)) & 3
+    so = nc
+    mo = so + T * ng * 2
+    ro = mo + T * ng * 2
+    s = rec[so:mo].view(np.float16).reshape(T, ng)
+    m = rec[mo:ro].view(np.float16).reshape(T, ng)
     r = rec[ro:ro + 2 * T].view(np.float16)
     c = rec[ro + 2 * T:ro + 2 * T + 2 * D].view(np.float16)
     pad = rec[ro + 2 * T + 2 * D:]
-    return dict(codes=codes.astype(np.uint8), s=gp[..., 0].copy(), m=gp[..., 1].copy(), r=r.copy(), c=c.copy(),
-                pad=pad.copy())
+    return dict(codes=codes.astype(np.uint8), s=s.copy(), m=m.copy(), r=r.copy(), c=c.copy(), pad=pad.copy())
 
 
 def near_f16_midpoint(x) -> np.ndarray:
@@ -55,9 +74,9 @@ def near_boundary(v, s) -> np.ndarray:
                                                        axis=-1) > 0)
 
 
-def check_block(rec, dbg: dict | None, oq: dict, T: int, D: int) -> dict:
+def check_block(rec, dbg: dict | None, oq: dict, T: int, D: int, layout: int) -> dict:
     """Compare one GPU record (+ optional fp32 debug scales) against an oracle quantize_block result."""
-    g = view_record(rec, T, D)
+    g = view_record(rec, T, D, layout)
     stats = dict(elements=T * D, boundary=0, code_flips=0, f16_flips=0)
     # codes
     nb = near_boundary(oq["v"], oq["s"])
@@ -91,7 +110,7 @@ def check_block(rec, dbg: dict | None, oq: dict, T: int, D: int) -> dict:
     return stats
 
 
-def oracle_records(x: np.ndarray, hb: int, sweeps: int = 4):
+def oracle_records(x: np.ndarray, hb: int, sweeps: int = 4, layout: int = oracle.K_ORDER):
     """Oracle quantisation of x [..., nblk*T, D] (float64) -> (records [..., nblk, rb], list of dicts)."""
     T = 128
     *lead, L, D = x.shape
@@ -102,7 +121,7 @@ def oracle_records(x: np.ndarray, hb: int, sweeps: int = 4):
     for i in range(flat.shape[0]):
         for b in range(nb):
             q = oracle.quantize_block(flat[i, b * T:(b + 1) * T], hb, sweeps)
-            recs[i, b] = oracle.pack_record(q)
+            recs[i, b] = oracle.pack_record(q, layout)
             qs.append(q)
     return recs.reshape(*lead, nb, -1), qs
 

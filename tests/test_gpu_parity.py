@@ -63,7 +63,8 @@ def test_quantize_blocks_matches_oracle(case):
                 for b in range(nb):
                     oq = oracle.quantize_block(xs[s, h, b * 128:(b + 1) * 128], hb, sweeps)
                     i = (s * H + h) * nb + b
-                    st = check_block(recs[s, h, 1 + b], {kk: dd[kk][i].numpy() for kk in "rcsm"}, oq, 128, D)
+                    st = check_block(recs[s, h, 1 + b], {kk: dd[kk][i].numpy() for kk in "rcsm"}, oq, 128, D,
+                                     oracle.V_ORDER if tensor else oracle.K_ORDER)
                     for kk in totals:
                         totals[kk] += st[kk]
     print(name, totals)
@@ -142,8 +143,8 @@ def _oracle_cache(cfg, k, v, L, hb, sweeps=4):
     krec = np.zeros((S, H, cfg.max_blocks, rb), dtype=np.uint8)
     vrec = np.zeros_like(krec)
     if nb:
-        krec[:, :, :nb] = oracle_records(kx, hb, sweeps)[0]
-        vrec[:, :, :nb] = oracle_records(vx, hb, sweeps)[0]
+        krec[:, :, :nb] = oracle_records(kx, hb, sweeps, oracle.K_ORDER)[0]
+        vrec[:, :, :nb] = oracle_records(vx, hb, sweeps, oracle.V_ORDER)[0]
     cache.k_records.copy_(torch.from_numpy(krec))
     cache.v_records.copy_(torch.from_numpy(vrec))
     cache.k_tail[:, :, :nt] = k[:, :, nb * 128:L].to(DEV)
@@ -251,8 +252,8 @@ def test_dequantize_matches_oracle(D, hb, dtype):
         ko, vo = ko.cpu().numpy(), vo.cpu().numpy()
         for h in range(H):
             for b in range(2):
-                for got, rec in ((ko, krec), (vo, vrec)):
-                    ref = oracle.dequantize_record(rec[0, h, b], 128, D, hb, rotated)
+                for got, rec, lay in ((ko, krec, oracle.K_ORDER), (vo, vrec, oracle.V_ORDER)):
+                    ref = oracle.dequantize_record(rec[0, h, b], 128, D, hb, rotated, lay)
                     np.testing.assert_allclose(got[0, h, b * 128:(b + 1) * 128], ref, rtol=2e-6,
                                                atol=2e-6 * np.abs(ref).max())
 
@@ -273,7 +274,9 @@ def test_closed_form_on_gpu():
     rms = math.sqrt(np.mean(b * b))
     np.testing.assert_allclose(dd["r"][0].numpy(), a * rms, rtol=1e-5)
     np.testing.assert_allclose(dd["c"][0].numpy(), b / rms, rtol=1e-5)
-    g = view_record(cache.k_records[0, 0, 0].cpu().numpy(), T, D)
+    g = view_record(cache.k_records[0, 0, 0].cpu().numpy(), T, D, oracle.K_ORDER)
+    np.testing.assert_array_equal(g["codes"], np.where(sign > 0, 3, 0))
+    g = view_record(cache.v_records[0, 0, 0].cpu().numpy(), T, D, oracle.V_ORDER)
     np.testing.assert_array_equal(g["codes"], np.where(sign > 0, 3, 0))
 
 
@@ -301,8 +304,8 @@ def test_power_of_two_token_scaling_is_exact_on_gpu():
     r[0, 5] *= 2.0 ** 6
     r[0, 90] *= 2.0 ** -4
     assert torch.equal(b["r"], r) and torch.equal(b["c"], a["c"]) and torch.equal(b["s"], a["s"])
-    ga = view_record(c1.k_records[0, 0, 0].cpu().numpy(), 128, 128)
-    gb = view_record(c2.k_records[0, 0, 0].cpu().numpy(), 128, 128)
+    ga = view_record(c1.k_records[0, 0, 0].cpu().numpy(), 128, 128, oracle.K_ORDER)
+    gb = view_record(c2.k_records[0, 0, 0].cpu().numpy(), 128, 128, oracle.K_ORDER)
     assert np.array_equal(ga["codes"], gb["codes"])
 
 
@@ -315,7 +318,8 @@ def test_zero_rows_on_gpu():
     dd = kvarn.debug_split(cfg, dk.cpu(), 1)
     assert float(dd["r"][0, 7]) == 1.0 and torch.all(dd["s"][0, 7] == 0)
     oq = oracle.quantize_block(to_f64(k[0, 0]), 128, 4)
-    check_block(cache.k_records[0, 0, 0].cpu().numpy(), {kk: dd[kk][0].numpy() for kk in "rcsm"}, oq, 128, 128)
+    check_block(cache.k_records[0, 0, 0].cpu().numpy(), {kk: dd[kk][0].numpy() for kk in "rcsm"}, oq, 128, 128,
+                oracle.K_ORDER)
 
 
 def test_kernels_are_deterministic():

@@ -205,14 +205,47 @@ def test_record_bit_layout():
     codes[0, :4] = [0, 1, 2, 3]
     codes[1, 4:8] = [3, 2, 1, 0]
     q = dict(codes=codes, r=np.full(T, 2.0), c=np.full(D, 0.5), s=np.full((T, 2), 0.25), m=np.full((T, 2), -1.0))
-    rec = oracle.pack_record(q)
-    assert len(rec) == oracle.record_bytes(T, D) == 3456  # 2048 + 1024 + 256 + 128, already 128-aligned
+    rec = oracle.pack_record(q, oracle.NATURAL)
+    assert len(rec) == oracle.record_bytes(T, D) == 3456  # 2048 + 512 + 512 + 256 + 128, already 128-aligned
     assert rec[0] == 0xE4 and rec[1] == 0 and rec[16 + 1] == 0x1B
-    g = np.frombuffer(rec[2048:2048 + 1024].tobytes(), dtype=np.float16).reshape(T, 2, 2)
-    assert np.all(g[..., 0] == 0.25) and np.all(g[..., 1] == -1.0)
+    assert np.all(np.frombuffer(rec[2048:2560].tobytes(), dtype=np.float16) == 0.25)
+    assert np.all(np.frombuffer(rec[2560:3072].tobytes(), dtype=np.float16) == -1.0)
     assert np.all(np.frombuffer(rec[3072:3328].tobytes(), dtype=np.float16) == 2.0)
     assert np.all(np.frombuffer(rec[3328:3456].tobytes(), dtype=np.float16) == 0.5)
     assert oracle.record_bytes(128, 128) == 6656 and oracle.record_bytes(128, 96) == 5120
+
+
+def _one_hot_site(layout, D, t, d):
+    """(word index, bit) where the code of (t, d) lands, found by packing a single 1."""
+    codes = np.zeros((128, D), dtype=np.uint8)
+    codes[t, d] = 1
+    q = dict(codes=codes, r=np.ones(128), c=np.ones(D), s=np.zeros((128, D // 32)), m=np.zeros((128, D // 32)))
+    words = oracle.pack_record(q, layout)[:32 * D].view(np.uint32)
+    (w,) = np.nonzero(words)
+    assert len(w) == 1
+    return int(w[0]), int(words[w[0]]).bit_length() - 1
+
+
+@pytest.mark.parametrize("layout", [oracle.K_ORDER, oracle.V_ORDER])
+@pytest.mark.parametrize("D", [64, 96, 128])
+def test_fragment_layouts_are_permutations_with_pairs(layout, D):
+    rng = np.random.default_rng(D + layout)
+    codes = rng.integers(0, 4, size=(128, D)).astype(np.uint8)
+    q = dict(codes=codes, r=np.ones(128), c=np.ones(D), s=np.ones((128, D // 32)), m=np.zeros((128, D // 32)))
+    rec = oracle.pack_record(q, layout)
+    np.testing.assert_array_equal(oracle.unpack_record(rec, 128, D, layout)["codes"], codes)
+    full = dict(q, codes=np.full((128, D), 3, dtype=np.uint8))
+    assert np.all(oracle.pack_record(full, layout)[:32 * D] == 0xFF)  # every code bit used exactly once
+    # the two codes an AND extracts as one binary16 pair sit at bit b and b + 16 of the same word:
+    # K pairs channels (k, k+1) of one token, V pairs tokens (t, t+1) of one channel
+    for t, d in [(0, 0), (37, 18), (127, D - 2), (64, 40), (90, 66 % D)]:
+        if layout == oracle.K_ORDER:
+            d -= d % 2
+            a, b = _one_hot_site(layout, D, t, d), _one_hot_site(layout, D, t, d + 1)
+        else:
+            t -= t % 2
+            a, b = _one_hot_site(layout, D, t, d), _one_hot_site(layout, D, t + 1, d)
+        assert a[0] == b[0] and b[1] == a[1] + 16 and a[1] < 16
 
 
 # ----------------------------------------------------------------- attention
