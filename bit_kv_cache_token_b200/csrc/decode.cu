@@ -21,12 +21,13 @@
 //   scores: A = q' (rows: query heads; hi/lo fp16 split in rows 0-7 / 8-15),
 //           B = K codes (k = channels, n = 8 tokens);
 //   P V:    A = p r s (rows: heads, hi/lo), B = V codes (k = tokens, n = 8 channels).
-// A 2-bit code becomes an exact fp16 operand with a single AND: the record
-// stores every code in a 32-bit word at bit 16*half + 2*pos (see kvarn.h),
-// so masking with 0x00030003 << 2*(pos%4) yields the pair as fp16 subnormals
-// c * 2^(2*(pos%4) - 24).  The 2^-(2*(pos%4)) part is folded into the other
-// operand (it depends only on the contracted index) and the remaining 2^-18
-// into the scales.  When the GQA group has fewer than 8 heads, the spare rows
+// A 2-bit code becomes an exact fp16 operand with a shift and an AND: the
+// record stores every code in a 32-bit word at bit 16*half + 2*pos (see
+// kvarn.h), and masking a shifted copy of the word puts both codes of a pair
+// on bits 8-9 or 6-7 of their halves, i.e. fp16 subnormals c * 2^-16 or
+// c * 2^-18.  The factor 4 between the two is folded into the other operand
+// (it depends only on the contracted index), the remaining 2^-16 into the
+// scales.  When the GQA group has fewer than 8 heads, the spare rows
 // carry copies of the heads working on other channel groups, so every lane
 // does useful work.  The last warp of a (sequence, kv head) to finish,
 // found with an atomic ticket, combines; no warp ever waits for another.
@@ -38,8 +39,8 @@
 namespace kvarn {
 
 constexpr int kDecWarps = 6;
-constexpr float kTwo18 = 262144.f;          // 2^18
-constexpr float kTwoM18 = 1.f / 262144.f;   // 2^-18
+constexpr float kTwo16 = 65536.f;           // 2^16
+constexpr float kTwoM16 = 1.f / 65536.f;    // 2^-16
 constexpr long long kWaitLimit = 1LL << 26; // bounded mbarrier polling
 
 template <int D, int GRP>
@@ -64,20 +65,51 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// fp32 pair -> (hi, lo) fp16 pairs with hi + lo = x to about 2^-22 relative.
+// fp32 pair -> fp16 pairs (hi, lo) with x = hi + lo * 2^-11 to about 2^-22
+// relative.  The remainder is scaled up by 2^11 so that it stays a normal
+// fp16 number whenever hi is; the MMA result of the lo rows is scaled back.
+constexpr float kLoUp = 2048.f;
+constexpr float kLoDown = 1.f / 2048.f;
 __device__ __forceinline__ void split_hilo(float x, float y, uint32_t &hi, uint32_t &lo)
 {
     const __half2 h = __floats2half2_rn(x, y);
     const float2 hf = __half22float2(h);
-    const __half2 l = __floats2half2_rn(x - hf.x, y - hf.y);
+    const __half2 l = __floats2half2_rn((x - hf.x) * kLoUp, (y - hf.y) * kLoUp);
     hi = *reinterpret_cast<const uint32_t *>(&h);
     lo = *reinterpret_cast<const uint32_t *>(&l);
 }
 
-// Two codes at position pos of word w as an fp16 pair (subnormal values).
-__device__ __forceinline__ uint32_t code_pair(uint32_t w, uint32_t w8, int pos)
+// hi rows (c0, c1) plus lo rows (c2, c3) of an accumulator
+__device__ __forceinline__ float2 hilo_sum(const float (&c)[4])
 {
-    return pos < 4 ? (w & (0x00030003u << (2 * pos))) : (w8 & (0x00030003u << (2 * (pos - 4))));
+    return f2(fmaf(c[2], kLoDown, c[0]), fmaf(c[3], kLoDown, c[1]));
+}
+
+// The five shifted copies of a code word from which every position is one AND.
+struct CodeWord {
+    uint32_t l8, l4, w, r4, r8;
+    __device__ __forceinline__ explicit CodeWord(uint32_t x) : l8(x << 8), l4(x << 4), w(x), r4(x >> 4), r8(x >> 8) {}
+    __device__ __forceinline__ CodeWord() : l8(0), l4(0), w(0), r4(0), r8(0) {}
+};
+
+// Two codes at position pos (0..7) of a word as an fp16 pair.  The code bits
+// land on bits 8-9 (even pos: value c * 2^-16) or 6-7 (odd pos: c * 2^-18) of
+// each half: the largest fp16 subnormals.  Smaller subnormal encodings lose
+// accumulation precision in the tensor core, whose alignment goes by the
+// encoded exponent.
+__device__ __forceinline__ uint32_t code_pair(const CodeWord &c, int pos)
+{
+    constexpr uint32_t kEven = 0x03000300u, kOdd = 0x00C000C0u;
+    switch (pos) {
+    case 0: return c.l8 & kEven;
+    case 1: return c.l4 & kOdd;
+    case 2: return c.l4 & kEven;
+    case 3: return c.w & kOdd;
+    case 4: return c.w & kEven;
+    case 5: return c.r4 & kOdd;
+    case 6: return c.r4 & kEven;
+    default: return c.r8 & kOdd;
+    }
 }
 
 __device__ __forceinline__ void mbar_init(unsigned long long *bar)
@@ -217,12 +249,12 @@ decode_kernel(DecodeArgs a, int hb)
         const unsigned char *vrec = sm.rec[stage][1];
         float *scr = sm.scr;
 
-        // ---- K scales to fp32: sK[g][t] = s * 2^18, rK[t], cK[d]
+        // ---- K scales to fp32: sK[g][t] = s * 2^16, rK[t], cK[d]
         {
             const __half *sh = reinterpret_cast<const __half *>(krec + R::kSOff);
             for (int idx = lane; idx < NG * kBlockTokens; idx += 32) {
                 const int t = idx / NG, g = idx % NG;
-                scr[g * kBlockTokens + t] = __half2float(sh[idx]) * kTwo18;
+                scr[g * kBlockTokens + t] = __half2float(sh[idx]) * kTwo16;
             }
             const __half *rh = reinterpret_cast<const __half *>(krec + R::kROff);
             for (int t = lane; t < kBlockTokens; t += 32) scr[NG * kBlockTokens + t] = __half2float(rh[t]);
@@ -245,12 +277,11 @@ decode_kernel(DecodeArgs a, int hb)
             Qg[kt / 2] += (v0 + v1) + (v2 + v3);
             const int g = kt / 2;
             const bool mine = (g % C) == copy;
-            // fold the code scale 2^(2*(q%4)) of channel block q = k/8 into q'
-            const float e0 = (kt & 1) ? 4.f : 64.f;   // q = 2kt
-            const float e1 = (kt & 1) ? 1.f : 16.f;   // q = 2kt + 1
+            // channel block q = 2kt + cs sits at an even position for cs = 0
+            // (code scale 2^-16) and an odd one for cs = 1 (2^-18): times 4
             if (mine) {
-                split_hilo(v0 * e0, v1 * e0, Aq[kt][0], Aq[kt][1]);
-                split_hilo(v2 * e1, v3 * e1, Aq[kt][2], Aq[kt][3]);
+                split_hilo(v0, v1, Aq[kt][0], Aq[kt][1]);
+                split_hilo(v2 * 4.f, v3 * 4.f, Aq[kt][2], Aq[kt][3]);
             } else {
                 Aq[kt][0] = Aq[kt][1] = Aq[kt][2] = Aq[kt][3] = 0u;
             }
@@ -275,13 +306,10 @@ decode_kernel(DecodeArgs a, int hb)
         float2 sc[16];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            uint32_t kw[KW], kw8[KW];
+            CodeWord kw[KW];
             const uint32_t *wp = reinterpret_cast<const uint32_t *>(krec) + (u * 32 + lane) * KW;
 #pragma unroll
-            for (int w = 0; w < KW; ++w) {
-                kw[w] = wp[w];
-                kw8[w] = kw[w] >> 8;
-            }
+            for (int w = 0; w < KW; ++w) kw[w] = CodeWord(wp[w]);
 #pragma unroll
             for (int ntl = 0; ntl < 2; ++ntl) {
                 const int nt8 = 2 * u + ntl;
@@ -297,7 +325,7 @@ decode_kernel(DecodeArgs a, int hb)
                         int word, pos;
                         if (q < 8 * F) { word = ntl * F + q / 8; pos = q % 8; }
                         else { word = 2 * F; pos = q - 8 * F + 4 * ntl; }
-                        bb[cs] = code_pair(kw[word], kw8[word], pos);
+                        bb[cs] = code_pair(kw[word], pos);
                     }
                     mma16816(acc[(kt / 2) / C], Aq[kt], bb[0], bb[1]);
                 }
@@ -311,12 +339,12 @@ decode_kernel(DecodeArgs a, int hb)
                     mma16816(accM, AM, *reinterpret_cast<uint32_t *>(&mp), 0u);
                 }
                 const int t0 = 8 * nt8 + 2 * tig;
-                float2 sum = f2(accM[0] + accM[2], accM[1] + accM[3]);
+                float2 sum = hilo_sum(accM);
 #pragma unroll
                 for (int st = 0; st < SETS; ++st) {
                     const int g = st * C + copy;
                     if (g < NG) {
-                        const float2 P = f2(acc[st][0] + acc[st][2], acc[st][1] + acc[st][3]);
+                        const float2 P = hilo_sum(acc[st]);
                         const float2 sp = *reinterpret_cast<const float2 *>(sK + g * kBlockTokens + t0);
                         sum = __ffma2_rn(P, sp, sum);
                     }
@@ -349,17 +377,19 @@ decode_kernel(DecodeArgs a, int hb)
         m_run = mnew;
         __syncwarp();  // every lane is done with the K scales
 
-        // ---- V scales: rsV[g][t] = r^V_t s^V_{t,g}, rV[t], cV[d] * 2^18
+        // ---- V scales: rsV[g][t] = r^V_t s^V_{t,g} e(t), rV[t], cV[d] * 2^16
         {
             const __half *sh = reinterpret_cast<const __half *>(vrec + R::kSOff);
             const __half *rh = reinterpret_cast<const __half *>(vrec + R::kROff);
             for (int idx = lane; idx < NG * kBlockTokens; idx += 32) {
                 const int t = idx / NG, g = idx % NG;
-                scr[g * kBlockTokens + t] = __half2float(sh[idx]) * __half2float(rh[t]);
+                // tokens t with odd t/32 sit at odd code positions (scale 2^-18): times 4
+                const float e = ((t >> 5) & 1) ? 4.f : 1.f;
+                scr[g * kBlockTokens + t] = __half2float(sh[idx]) * __half2float(rh[t]) * e;
             }
             for (int t = lane; t < kBlockTokens; t += 32) scr[NG * kBlockTokens + t] = __half2float(rh[t]);
             const __half *ch = reinterpret_cast<const __half *>(vrec + R::kCOff);
-            for (int d = lane; d < D; d += 32) scr[(NG + 1) * kBlockTokens + d] = __half2float(ch[d]) * kTwo18;
+            for (int d = lane; d < D; d += 32) scr[(NG + 1) * kBlockTokens + d] = __half2float(ch[d]) * kTwo16;
         }
         __syncwarp();
         const float *rsV = scr, *rV = scr + NG * kBlockTokens, *cV = scr + (NG + 1) * kBlockTokens;
@@ -386,7 +416,7 @@ decode_kernel(DecodeArgs a, int hb)
                 mma16816(accB, Ab, bb0, bb1);
             }
         }
-        const float2 bpair = f2(accB[0] + accB[2], accB[1] + accB[3]);  // (h, groups 2tig, 2tig+1)
+        const float2 bpair = hilo_sum(accB);  // (h, groups 2tig, 2tig+1)
 
         // ---- P V, one group set at a time
 #pragma unroll
@@ -400,11 +430,11 @@ decode_kernel(DecodeArgs a, int hb)
             for (int ks = 0; ks < 8; ++ks) {
                 const int T0 = 16 * ks + 2 * tig, T1 = T0 + 8;
                 if (gv) {
-                    const float e = (ks >> 1) == 0 ? 64.f : (ks >> 1) == 1 ? 16.f : (ks >> 1) == 2 ? 4.f : 1.f;
                     const float2 r0 = *reinterpret_cast<const float2 *>(rsV + g * kBlockTokens + T0);
                     const float2 r1 = *reinterpret_cast<const float2 *>(rsV + g * kBlockTokens + T1);
-                    split_hilo(sc[2 * ks].x * r0.x * e, sc[2 * ks].y * r0.y * e, Av[ks][0], Av[ks][1]);
-                    split_hilo(sc[2 * ks + 1].x * r1.x * e, sc[2 * ks + 1].y * r1.y * e, Av[ks][2], Av[ks][3]);
+                    const float2 p0 = __fmul2_rn(sc[2 * ks], r0), p1 = __fmul2_rn(sc[2 * ks + 1], r1);
+                    split_hilo(p0.x, p0.y, Av[ks][0], Av[ks][1]);
+                    split_hilo(p1.x, p1.y, Av[ks][2], Av[ks][3]);
                 } else {
                     Av[ks][0] = Av[ks][1] = Av[ks][2] = Av[ks][3] = 0u;
                 }
@@ -413,7 +443,7 @@ decode_kernel(DecodeArgs a, int hb)
             const int gsrc = gv ? g : 0;
             const float bx = __shfl_sync(0xffffffffu, bpair.x, 4 * h + gsrc / 2);
             const float by = __shfl_sync(0xffffffffu, bpair.y, 4 * h + gsrc / 2);
-            const float bias = ((gsrc & 1) ? by : bx) * kTwoM18;
+            const float bias = ((gsrc & 1) ? by : bx) * kTwoM16;
 #pragma unroll
             for (int cc = 0; cc < C; ++cc) {
                 const int gg = st * C + cc;
@@ -422,7 +452,7 @@ decode_kernel(DecodeArgs a, int hb)
                 for (int j4 = 0; j4 < kGroup / 8; ++j4) {
                     const int nt = gg * (kGroup / 8) + j4;
                     const uint2 vw2 = reinterpret_cast<const uint2 *>(vrec)[nt * 32 + lane];
-                    const uint32_t vw[2] = {vw2.x, vw2.y}, vw8[2] = {vw2.x >> 8, vw2.y >> 8};
+                    const CodeWord vw[2] = {CodeWord(vw2.x), CodeWord(vw2.y)};
                     float acc4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
@@ -430,13 +460,14 @@ decode_kernel(DecodeArgs a, int hb)
 #pragma unroll
                         for (int cs = 0; cs < 2; ++cs) {
                             const int m = 2 * ks + cs, am = m % 4;
-                            bb[cs] = code_pair(vw[am / 2], vw8[am / 2], 4 * (am % 2) + m / 4);
+                            bb[cs] = code_pair(vw[am / 2], 4 * (am % 2) + m / 4);
                         }
                         mma16816(acc4, Av[ks], bb[0], bb[1]);
                     }
                     if (cc == copy) {
                         const float2 cv = *reinterpret_cast<const float2 *>(cV + 8 * nt + 2 * tig);
-                        const float2 o = f2(acc4[0] + acc4[2] + bias, acc4[1] + acc4[3] + bias);
+                        const float2 hs = hilo_sum(acc4);
+                        const float2 o = f2(hs.x + bias, hs.y + bias);
                         orun[nt] = __ffma2_rn(o, cv, orun[nt]);
                     }
                 }
