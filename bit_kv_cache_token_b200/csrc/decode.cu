@@ -15,8 +15,10 @@
 //
 // B200 mapping.  One warp streams a contiguous range of 128-token blocks of
 // one (sequence, kv head) with its own online softmax; the records reach
-// shared memory by cp.async.bulk (TMA) into a two-stage ring guarded by
-// mbarriers.  Both contractions run on tensor cores (mma.sync m16n8k16, fp16
+// shared memory by cp.async.bulk (TMA), one buffer each for K and V guarded
+// by mbarriers: the next K record is requested as soon as the scores are
+// done, the next V record as soon as P V is done, so each copy overlaps half
+// a block of this warp's work and the whole work of the SM's other warps.  Both contractions run on tensor cores (mma.sync m16n8k16, fp16
 // in, fp32 accumulate):
 //   scores: A = q' (rows: query heads; hi/lo fp16 split in rows 0-7 / 8-15),
 //           B = K codes (k = channels, n = 8 tokens);
@@ -38,18 +40,25 @@
 
 namespace kvarn {
 
-constexpr int kDecWarps = 6;
 constexpr float kTwo16 = 65536.f;           // 2^16
 constexpr float kTwoM16 = 1.f / 65536.f;    // 2^-16
 constexpr long long kWaitLimit = 1LL << 26; // bounded mbarrier polling
 
 template <int D, int GRP>
 struct alignas(128) DecWarpSmem {
-    unsigned char rec[2][2][Record<D>::kBytes];  // [stage][K, V]
+    unsigned char rec[2][Record<D>::kBytes];  // [K, V] of the current block
     float scr[(D / kGroup) * kBlockTokens + kBlockTokens + D];
     float qbuf[GRP][D];
-    unsigned long long mbar[2];
+    unsigned long long mbar[2];               // K record, V record
 };
+
+// Warps per CTA: up to 12, as many as fit in 227 KB of shared memory.
+template <int D, int GRP>
+__host__ __device__ constexpr int dec_warps()
+{
+    constexpr int fit = (227 * 1024) / (int)sizeof(DecWarpSmem<D, GRP>);
+    return fit < 12 ? fit : 12;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -118,20 +127,16 @@ __device__ __forceinline__ void mbar_init(unsigned long long *bar)
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
 }
 
-// Lane 0 only: stage both records of block b (K then V) into stage buffers.
-__device__ __forceinline__ void issue_block(unsigned long long *bar, unsigned char *kdst, unsigned char *vdst,
-                                            const unsigned char *ksrc, const unsigned char *vsrc, uint32_t bytes)
+// Lane 0 only: stage one record (bytes, multiple of 16) into shared memory.
+__device__ __forceinline__ void issue_record(unsigned long long *bar, unsigned char *dst, const unsigned char *src,
+                                             uint32_t bytes)
 {
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(2 * bytes)
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-                     smem_u32(kdst)),
-                 "l"(ksrc), "r"(bytes), "r"(smem_u32(bar))
-                 : "memory");
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-                     smem_u32(vdst)),
-                 "l"(vsrc), "r"(bytes), "r"(smem_u32(bar))
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
 }
 
@@ -174,7 +179,7 @@ __device__ void warp_fwht(float *x, int nvec, int hb)
 }
 
 template <int D, int GRP, typename Tin>
-__global__ void __launch_bounds__(kDecWarps * 32, 1)
+__global__ void __launch_bounds__(dec_warps<D, GRP>() * 32, 1)
 decode_kernel(DecodeArgs a, int hb)
 {
     using R = Record<D>;
@@ -189,7 +194,7 @@ decode_kernel(DecodeArgs a, int hb)
     extern __shared__ __align__(128) unsigned char smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     DecWarpSmem<D, GRP> &sm = reinterpret_cast<DecWarpSmem<D, GRP> *>(smem_raw)[warp];
-    const int item = blockIdx.x * kDecWarps + warp;
+    const int item = blockIdx.x * dec_warps<D, GRP>() + warp;
     const int nitems = a.num_units * a.nsplit;
     if (item >= nitems) return;
     const int unit = item / a.nsplit, split = item % a.nsplit;
@@ -213,15 +218,6 @@ decode_kernel(DecodeArgs a, int hb)
     for (int i = lane; i < GRP * D; i += 32) (&sm.qbuf[0][0])[i] = In<Tin>::load1(qg + i) * a.scale_log2;
     __syncwarp();
     warp_fwht<D>(&sm.qbuf[0][0], GRP, hb);
-    float qreg[NKT][4];  // q_rot at channels 16kt + 2tig + {0, 1, 8, 9}
-#pragma unroll
-    for (int kt = 0; kt < NKT; ++kt) {
-        const int k = 16 * kt + 2 * tig;
-        qreg[kt][0] = sm.qbuf[h][k];
-        qreg[kt][1] = sm.qbuf[h][k + 1];
-        qreg[kt][2] = sm.qbuf[h][k + 8];
-        qreg[kt][3] = sm.qbuf[h][k + 9];
-    }
 
     float m_run = -INFINITY, l_run = 0.f;
     float2 orun[NNT];
@@ -236,17 +232,16 @@ decode_kernel(DecodeArgs a, int hb)
         mbar_init(&sm.mbar[1]);
     }
     __syncwarp();
-    if (lane == 0) {
-        for (int i = 0; i < 2 && b0 + i < b1; ++i)
-            issue_block(&sm.mbar[i], sm.rec[i][0], sm.rec[i][1], kbase + (size_t)(b0 + i) * R::kBytes,
-                        vbase + (size_t)(b0 + i) * R::kBytes, R::kBytes);
+    if (lane == 0 && b0 < b1) {
+        issue_record(&sm.mbar[0], sm.rec[0], kbase + (size_t)b0 * R::kBytes, R::kBytes);
+        issue_record(&sm.mbar[1], sm.rec[1], vbase + (size_t)b0 * R::kBytes, R::kBytes);
     }
 
     for (int b = b0; b < b1; ++b) {
-        const int i = b - b0, stage = i & 1;
-        if (!mbar_wait(&sm.mbar[stage], (i >> 1) & 1)) { failed_at = i; break; }
-        const unsigned char *krec = sm.rec[stage][0];
-        const unsigned char *vrec = sm.rec[stage][1];
+        const int i = b - b0;
+        if (!mbar_wait(&sm.mbar[0], i & 1)) { failed_at = i; break; }
+        const unsigned char *krec = sm.rec[0];
+        const unsigned char *vrec = sm.rec[1];
         float *scr = sm.scr;
 
         // ---- K scales to fp32: sK[g][t] = s * 2^16, rK[t], cK[d]
@@ -272,8 +267,10 @@ decode_kernel(DecodeArgs a, int hb)
 #pragma unroll
         for (int kt = 0; kt < NKT; ++kt) {
             const int k = 16 * kt + 2 * tig;
-            const float v0 = qreg[kt][0] * cK[k], v1 = qreg[kt][1] * cK[k + 1];
-            const float v2 = qreg[kt][2] * cK[k + 8], v3 = qreg[kt][3] * cK[k + 9];
+            const float2 q01 = *reinterpret_cast<const float2 *>(&sm.qbuf[h][k]);
+            const float2 q89 = *reinterpret_cast<const float2 *>(&sm.qbuf[h][k + 8]);
+            const float v0 = q01.x * cK[k], v1 = q01.y * cK[k + 1];
+            const float v2 = q89.x * cK[k + 8], v3 = q89.y * cK[k + 9];
             Qg[kt / 2] += (v0 + v1) + (v2 + v3);
             const int g = kt / 2;
             const bool mine = (g % C) == copy;
@@ -375,7 +372,10 @@ decode_kernel(DecodeArgs a, int hb)
         }
         l_run = fmaf(l_run, alpha, ls);
         m_run = mnew;
-        __syncwarp();  // every lane is done with the K scales
+        __syncwarp();  // every lane is done with the K record and the K scales
+        if (lane == 0 && b + 1 < b1)
+            issue_record(&sm.mbar[0], sm.rec[0], kbase + (size_t)(b + 1) * R::kBytes, R::kBytes);
+        if (!mbar_wait(&sm.mbar[1], i & 1)) { failed_at = i; break; }
 
         // ---- V scales: rsV[g][t] = r^V_t s^V_{t,g} e(t), rV[t], cV[d] * 2^16
         {
@@ -474,16 +474,19 @@ decode_kernel(DecodeArgs a, int hb)
             }
         }
 
-        // ---- refill this stage with block b + 2
+        // ---- the V buffer is free: request the next V record
         __syncwarp();
-        if (lane == 0 && b + 2 < b1)
-            issue_block(&sm.mbar[stage], sm.rec[stage][0], sm.rec[stage][1], kbase + (size_t)(b + 2) * R::kBytes,
-                        vbase + (size_t)(b + 2) * R::kBytes, R::kBytes);
+        if (lane == 0 && b + 1 < b1)
+            issue_record(&sm.mbar[1], sm.rec[1], vbase + (size_t)(b + 1) * R::kBytes, R::kBytes);
     }
     if (failed_at >= 0) {
         // let the copies this warp may still have in flight land (bounded), then report
         if (lane == 0) {
-            for (int i = failed_at; i < failed_at + 2 && i < b1 - b0; ++i) mbar_wait(&sm.mbar[i & 1], (i >> 1) & 1);
+            // at most one copy per buffer can be outstanding: the one of block failed_at
+            // (or of failed_at + 1 for K when the V wait gave up)
+            mbar_wait(&sm.mbar[0], failed_at & 1);
+            if (failed_at + 1 < b1 - b0) mbar_wait(&sm.mbar[0], (failed_at + 1) & 1);
+            mbar_wait(&sm.mbar[1], failed_at & 1);
             status_or(a.status, KVARN_STATUS_TIMEOUT);
         }
         __syncwarp();
@@ -591,8 +594,8 @@ decode_kernel(DecodeArgs a, int hb)
     if (lane == 0) a.tickets[unit] = 0u;
     __threadfence();
 
-    float *obuf = reinterpret_cast<float *>(sm.rec[0][0]);   // [GRP][D] rotated part
-    float *otl = reinterpret_cast<float *>(sm.rec[1][0]);    // [GRP][D] tail part
+    float *obuf = reinterpret_cast<float *>(sm.rec[0]);   // [GRP][D] rotated part
+    float *otl = reinterpret_cast<float *>(sm.rec[1]);    // [GRP][D] tail part
     for (int hh = 0; hh < GRP; ++hh) {
         float M = -INFINITY;
         for (int i = 0; i <= a.nsplit; ++i) M = fmaxf(M, __ldcg(pbase + ((size_t)i * GRP + hh) * (D + 2)));
@@ -628,13 +631,14 @@ decode_kernel(DecodeArgs a, int hb)
 template <int D, int GRP, typename Tin>
 static cudaError_t launch_dec(const DecodeArgs &a, int hb, cudaStream_t st)
 {
-    const size_t smem = sizeof(DecWarpSmem<D, GRP>) * kDecWarps;
+    constexpr int W = dec_warps<D, GRP>();
+    const size_t smem = sizeof(DecWarpSmem<D, GRP>) * W;
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, GRP, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     const int items = a.num_units * a.nsplit;
-    dim3 grid((unsigned)((items + kDecWarps - 1) / kDecWarps));
-    decode_kernel<D, GRP, Tin><<<grid, kDecWarps * 32, smem, st>>>(a, hb);
+    dim3 grid((unsigned)((items + W - 1) / W));
+    decode_kernel<D, GRP, Tin><<<grid, W * 32, smem, st>>>(a, hb);
     return cudaGetLastError();
 }
 
@@ -666,6 +670,20 @@ cudaError_t run_decode(const kvarn_config &c, const DecodeArgs &a, cudaStream_t 
     return cudaErrorInvalidValue;
 }
 
-int decode_warps_per_cta() { return kDecWarps; }
+template <int D>
+static int warps_for(int grp)
+{
+    switch (grp) {
+    case 1: return dec_warps<D, 1>();
+    case 2: return dec_warps<D, 2>();
+    case 4: return dec_warps<D, 4>();
+    default: return dec_warps<D, 8>();
+    }
+}
+
+int decode_warps_per_cta(int head_dim, int grp)
+{
+    return head_dim == 64 ? warps_for<64>(grp) : head_dim == 96 ? warps_for<96>(grp) : warps_for<128>(grp);
+}
 
 }  // namespace kvarn

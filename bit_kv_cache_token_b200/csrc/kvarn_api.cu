@@ -160,12 +160,12 @@ int kvarn_decode_attention(const kvarn_config *cfg, const void *q, int num_q_hea
     if (!workspace || !aligned16(workspace) || workspace_bytes < need) return KVARN_EWORKSPACE;
 
     // one warp per (sequence, kv head, split); splits sized so that all warps
-    // are resident at once (one CTA of decode_warps_per_cta() warps per SM)
+    // are resident at once (one CTA of decode_warps_per_cta warps per SM)
     const int units = cfg->num_seqs * cfg->num_kv_heads;
     const int nblk = max_tokens / cfg->block_tokens;
     int nsplit = 1, bps = nblk > 0 ? nblk : 1;
     if (nblk > 0) {
-        int ns = num_sms() * decode_warps_per_cta() / units;
+        int ns = num_sms() * decode_warps_per_cta(cfg->head_dim, grp) / units;
         ns = ns < 1 ? 1 : ns;
         ns = ns > nblk ? nblk : ns;
         ns = ns > kMaxSplits ? kMaxSplits : ns;

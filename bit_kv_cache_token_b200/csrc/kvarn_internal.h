@@ -60,6 +60,6 @@ cudaError_t run_set_length(int32_t *n_tokens, int num_seqs, int value, cudaStrea
 constexpr int kMaxSplits = 64;
 
 // Warps per decode CTA (one CTA per SM by shared memory).
-int decode_warps_per_cta();
+int decode_warps_per_cta(int head_dim, int grp);
 
 }  // namespace kvarn

@@ -35,7 +35,8 @@ quantize_blocks_kernel(QuantArgs a)
                          slot * Record<D>::kBytes;
     float *dbg = tensor ? a.debug_v : a.debug_k;
     if (dbg) dbg += ((size_t)sh * nb + b) * (kBlockTokens + D + 2 * kBlockTokens * (D / kGroup));
-    quantize_block<D, HB>(X, sm, a.sweeps, tensor, rec, dbg, a.status);
+    if (tensor) quantize_block<D, HB, 1>(X, sm, a.sweeps, rec, dbg, a.status);
+    else quantize_block<D, HB, 0>(X, sm, a.sweeps, rec, dbg, a.status);
 }
 
 // One CTA per (sequence, kv head) and per tensor.  The token goes into tail
@@ -68,7 +69,8 @@ append_kernel(AppendArgs a)
             load_block<D>(tail, X);
             unsigned char *rec = static_cast<unsigned char *>(tensor ? a.v_records : a.k_records) +
                                  ((size_t)sh * a.max_blocks + blk) * Record<D>::kBytes;
-            quantize_block<D, HB>(X, sm, a.sweeps, tensor, rec, nullptr, a.status);
+            if (tensor) quantize_block<D, HB, 1>(X, sm, a.sweeps, rec, nullptr, a.status);
+            else quantize_block<D, HB, 0>(X, sm, a.sweeps, rec, nullptr, a.status);
         }
     } else if (threadIdx.x == 0 && tensor == 0 && (sh % a.num_kv_heads) == 0) {
         status_or(a.status, KVARN_STATUS_CAPACITY);

@@ -31,7 +31,7 @@ template <int D>
 struct QuantSmem {
     static constexpr int W = D / 32;
     union {
-        float xch[W][32][32];                  // Hadamard exchange [warp][i][lane]
+        float4 xch[W][2][8][32];               // Hadamard exchange [warp][token pair][chunk][lane]
         float4 col[W][32][16];                 // column-sum transpose [warp][lane][chunk]
         unsigned char rec[Record<D>::kBytes];  // record staging
     } u;
@@ -40,6 +40,20 @@ struct QuantSmem {
 };
 
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, f2(-1.f, -1.f), a); }
+
+__device__ __forceinline__ float min3(float a, float b, float c)
+{
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
 
 // In-register 32-point Walsh-Hadamard butterflies (unnormalised) on one token.
 __device__ __forceinline__ void fwht32_regs(float2 (&x)[16])
@@ -81,10 +95,10 @@ __device__ __forceinline__ void load_block(const Tin *rows, float2 (&X)[4][16])
 }
 
 // Quantise the block held in X (destroyed) into rec_out (global, 16-byte
-// aligned, Record<D>::kBytes); tensor 0 = K code order, 1 = V code order.  dbg: NULL or fp32 [T + D + 2*T*D/32] unrounded
+// aligned, Record<D>::kBytes); TENSOR 0 = K code order, 1 = V code order.  dbg: NULL or fp32 [T + D + 2*T*D/32] unrounded
 // r, c, s, m.  All D threads of the CTA must call this.
-template <int D, int HB>
-__device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps, int tensor,
+template <int D, int HB, int TENSOR>
+__device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
                                unsigned char *__restrict__ rec_out, float *__restrict__ dbg,
                                int32_t *status)
 {
@@ -97,28 +111,30 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
 #pragma unroll
         for (int r = 0; r < 4; ++r) fwht32_regs(X[r]);
         if constexpr (HB > 32) {
-            constexpr int M = HB / 32;  // warps per Hadamard block
-            const int jj = j % M, jb = j - jj;
+            // the remaining butterflies pair warps j and j ^ m (channel bit 5 + log2 m),
+            // one stage per bit, two tokens at a time through shared memory
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
+            for (int m = 1; m < HB / 32; m <<= 1) {
+                const float sg = (j & m) ? -1.f : 1.f;  // upper half of the pair: partner - own
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    sm.u.xch[j][2 * k][l] = X[r][k].x;
-                    sm.u.xch[j][2 * k + 1][l] = X[r][k].y;
+                for (int rp = 0; rp < 4; rp += 2) {
+#pragma unroll
+                    for (int r = 0; r < 2; ++r)
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            sm.u.xch[j][r][q][l] = make_float4(X[rp + r][2 * q].x, X[rp + r][2 * q].y,
+                                                               X[rp + r][2 * q + 1].x, X[rp + r][2 * q + 1].y);
+                    __syncthreads();
+#pragma unroll
+                    for (int r = 0; r < 2; ++r)
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 p = sm.u.xch[j ^ m][r][q][l];
+                            X[rp + r][2 * q] = __ffma2_rn(f2(sg, sg), X[rp + r][2 * q], f2(p.x, p.y));
+                            X[rp + r][2 * q + 1] = __ffma2_rn(f2(sg, sg), X[rp + r][2 * q + 1], f2(p.z, p.w));
+                        }
+                    __syncthreads();
                 }
-                __syncthreads();
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    float2 acc = f2(0.f, 0.f);
-#pragma unroll
-                    for (int m = 0; m < M; ++m) {
-                        const float sgn = (__popc(jj & m) & 1) ? -1.f : 1.f;
-                        const float2 v = f2(sm.u.xch[jb + m][2 * k][l], sm.u.xch[jb + m][2 * k + 1][l]);
-                        acc = __ffma2_rn(f2(sgn, sgn), v, acc);
-                    }
-                    X[r][k] = acc;
-                }
-                __syncthreads();
             }
         }
         const float nrm = HB == 32 ? 0.17677669529663688f : HB == 64 ? 0.125f : 0.08838834764831845f;  // 1/sqrt(HB)
@@ -161,13 +177,8 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
             }
             const float mean = S1 * (1.f / D);
             const float var = fmaf(-mean, mean, S2 * (1.f / D));
-            if (var > 0.f) {
-                rt[r] = sqrtf(var);
-                w[r] = 1.f / rt[r];
-            } else {
-                rt[r] = 1.f;
-                w[r] = 1.f;
-            }
+            w[r] = var > 0.f ? rsqrtf(var) : 1.f;  // 1 / r_t
+            rt[r] = var > 0.f ? var * w[r] : 1.f;  // r_t = sqrt(var)
         }
         // column step: c_d = std over the 128 tokens of X / r
 #pragma unroll
@@ -198,9 +209,10 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
             }
             const float mean = acc.x * (1.f / kBlockTokens);
             const float var = fmaf(-mean, mean, acc.y * (1.f / kBlockTokens));
-            cd = var > 0.f ? sqrtf(var) : 1.f;
+            const float ud = var > 0.f ? rsqrtf(var) : 1.f;  // 1 / c_d
+            cd = var > 0.f ? var * ud : 1.f;
             __syncwarp();
-            sm.ubuf[32 * j + l] = 1.f / cd;
+            sm.ubuf[32 * j + l] = ud;
             __syncwarp();
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -218,7 +230,10 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
     // of one token fill one byte.  V: the codes of one channel for this
     // thread's 4 tokens (l + 32r) fill one byte.
     unsigned char *rec = sm.u.rec;
-    uint32_t vbytes[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // V: channel i in byte i%4 of vbytes[i/4]
+    // Codes are read from the low mantissa bits of lev = 1.5*2^23 + code, whose
+    // bit pattern is 0x4B400000 + code: multiply-adding the raw patterns with the
+    // code weights and subtracting the pattern's share once packs them.
+    uint32_t vacc[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // V: channel i in byte i%4 of vacc[i/4]
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         const int t = l + 32 * r;
@@ -227,8 +242,8 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
             z[k] = __fmul2_rn(X[r][k], u[k]);
-            mn = fminf(mn, fminf(z[k].x, z[k].y));
-            mx = fmaxf(mx, fmaxf(z[k].x, z[k].y));
+            mn = min3(mn, z[k].x, z[k].y);
+            mx = max3(mx, z[k].x, z[k].y);
         }
         const float range = mx - mn;
         // level = (Z - min) * 3 / range: Z = Y * r_t, so this equals (Y - m) / s
@@ -238,21 +253,27 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
         // 12582912 = 1.5 * 2^23: adding it rounds the level to an integer
         // (ties to even) and leaves that integer in the low mantissa bits.
         const float2 magic = f2(12582912.f, 12582912.f);
-        uint32_t kbytes[4] = {0u, 0u, 0u, 0u};  // K: byte (tig, half) at bits 8*half of kbytes[tig]
+        uint32_t kacc[4] = {0u, 0u, 0u, 0u};  // K: byte (tig, half) at bits 8*half of kacc[tig]
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
             const float2 lev = __fadd2_rn(__ffma2_rn(z[k], kq2, nmk), magic);
-            const uint32_t c0 = __float_as_uint(lev.x) & 3u, c1 = __float_as_uint(lev.y) & 3u;
-            // local channels 2k (c0) and 2k+1 (c1): x = k/4, tig = k%4
-            kbytes[k & 3] |= (c0 << (2 * (k >> 2))) | (c1 << (8 + 2 * (k >> 2)));
-            vbytes[k >> 1] |= (c0 << (16 * (k & 1) + 2 * r)) | (c1 << (16 * (k & 1) + 8 + 2 * r));
+            const uint32_t b0 = __float_as_uint(lev.x), b1 = __float_as_uint(lev.y);
+            // local channels 2k (b0) and 2k+1 (b1): x = k/4, tig = k%4
+            if constexpr (TENSOR == 0) {
+                kacc[k & 3] += b0 * (1u << (2 * (k >> 2))) + b1 * (1u << (8 + 2 * (k >> 2)));
+            } else {
+                vacc[k >> 1] += b0 * (1u << (16 * (k & 1) + 2 * r)) + b1 * (1u << (16 * (k & 1) + 8 + 2 * r));
+            }
         }
-        if (tensor == 0) {
+        if constexpr (TENSOR == 0) {
+            // remove 0x4B400000 * (1 + 4 + 16 + 64) * (1 + 256) from each word
+            constexpr uint32_t kBias = 0x4B400000u * 85u * 257u;
 #pragma unroll
             for (int tig = 0; tig < 4; ++tig) {
+                const uint32_t v = kacc[tig] - kBias;
                 const int kch = 32 * j + 2 * tig;  // channel with x = 0, half = 0
-                rec[k_code_bit<D>(t, kch) / 8] = (unsigned char)(kbytes[tig] & 0xFFu);
-                rec[k_code_bit<D>(t, kch + 1) / 8] = (unsigned char)(kbytes[tig] >> 8);
+                rec[k_code_bit<D>(t, kch) / 8] = (unsigned char)(v & 0xFFu);
+                rec[k_code_bit<D>(t, kch + 1) / 8] = (unsigned char)((v >> 8) & 0xFFu);
             }
         }
         const float s = range * w[r] * (1.f / 3.f);
@@ -273,10 +294,14 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
             dbg[kBlockTokens + D + kBlockTokens * (D / 32) + t * (D / 32) + j] = m;
         }
     }
-    if (tensor == 1) {
+    if constexpr (TENSOR == 1) {
+        // each vacc word took 0x4B400000 * (1 + 4 + 16 + 64) * (1 + 256 + 65536 + 2^24)
+        constexpr uint32_t kBias = 0x4B400000u * 85u * 16843009u;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) vacc[q] -= kBias;
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-            rec[v_code_bit(l, 32 * j + i) / 8] = (unsigned char)(vbytes[i >> 2] >> (8 * (i & 3)));
+            rec[v_code_bit(l, 32 * j + i) / 8] = (unsigned char)(vacc[i >> 2] >> (8 * (i & 3)));
     }
     {
         const __half hc = __float2half_rn(cd);
@@ -284,8 +309,9 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
         *reinterpret_cast<__half *>(rec + R::kCOff + 2 * (32 * j + l)) = hc;
         if (dbg) dbg[kBlockTokens + 32 * j + l] = cd;
     }
-    if (threadIdx.x < (R::kBytes - R::kRaw) / 4)  // zero the padding
-        reinterpret_cast<uint32_t *>(rec + R::kRaw)[threadIdx.x] = 0u;
+    if constexpr (R::kBytes > R::kRaw) {  // zero the padding
+        if (threadIdx.x < (R::kBytes - R::kRaw) / 4) reinterpret_cast<uint32_t *>(rec + R::kRaw)[threadIdx.x] = 0u;
+    }
     __syncthreads();
     // ---- 4. coalesced 16-byte copy of the record to global ---------------
     for (int i = threadIdx.x; i < R::kBytes / 16; i += D)
