@@ -31,6 +31,7 @@ KVARN_BF16 = 1
 EXPORTED = (
     "kvarn_record_bytes", "kvarn_cache_bytes", "kvarn_decode_workspace_bytes", "kvarn_quantize_blocks",
     "kvarn_append_token", "kvarn_decode_attention", "kvarn_dequantize", "kvarn_strerror",
+    "kvarn_decode_attention_noalloc",
 )
 
 
@@ -73,9 +74,11 @@ def lib() -> ctypes.CDLL:
         L.kvarn_append_token.argtypes = [P(kvarn_config), V, V, P(kvarn_cache), V]
         L.kvarn_decode_attention.argtypes = [P(kvarn_config), V, I, F, P(kvarn_cache), I, V, V, S, V]
         L.kvarn_dequantize.argtypes = [P(kvarn_config), P(kvarn_cache), I, I, I, V, V, V]
+        L.kvarn_decode_attention_noalloc.argtypes = [P(kvarn_config), V, I, F, P(kvarn_cache), I, V, V]
         L.kvarn_strerror.argtypes = [I]
         L.kvarn_strerror.restype = ctypes.c_char_p
-        for name in ("kvarn_quantize_blocks", "kvarn_append_token", "kvarn_decode_attention", "kvarn_dequantize"):
+        for name in ("kvarn_quantize_blocks", "kvarn_append_token", "kvarn_decode_attention", "kvarn_dequantize",
+                     "kvarn_decode_attention_noalloc"):
             getattr(L, name).restype = I
         _lib = L
     return _lib
@@ -228,6 +231,20 @@ def decode_attention(cfg: Config, q, cache: KVCache, max_tokens: int, out=None, 
     _check(lib().kvarn_decode_attention(ctypes.byref(c), _ptr(q), int(Hq), float(softmax_scale), ctypes.byref(cs),
                                         int(max_tokens), _ptr(out), _ptr(workspace), int(workspace.numel()),
                                         _stream(stream)), "kvarn_decode_attention")
+    return out
+
+
+def decode_attention_noalloc(cfg: Config, q, cache: KVCache, max_tokens: int, out, softmax_scale: float = 0.0,
+                             stream=None):
+    """kvarn_decode_attention_noalloc: like decode_attention, with the library's own static workspace.
+
+    `out` must be given (this path allocates nothing); calls that overlap on the GPU race."""
+    _need(q, "q", cfg.torch_dtype)
+    _need(out, "out", torch.float32)
+    c, cs = cfg.c(), cache.struct()
+    _check(lib().kvarn_decode_attention_noalloc(ctypes.byref(c), _ptr(q), int(q.shape[1]), float(softmax_scale),
+                                                ctypes.byref(cs), int(max_tokens), _ptr(out), _stream(stream)),
+           "kvarn_decode_attention_noalloc")
     return out
 
 

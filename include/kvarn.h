@@ -203,6 +203,27 @@ KVARN_API int kvarn_decode_attention(const kvarn_config *cfg, const void *q, int
 KVARN_API int kvarn_dequantize(const kvarn_config *cfg, const kvarn_cache *cache, int first_block,
                      int num_blocks, int rotated, float *k_out, float *v_out, void *stream);
 
+/*
+ * kvarn_decode_attention without a workspace argument, for callers that
+ * cannot allocate device memory where they run decode (code running inside a
+ * host callback or another runtime's allocator, or a process that must not
+ * grow its device footprint after start-up).  There is no counterpart on the
+ * pages: this is a deployment variant of the same kernel.
+ * The workspace is a 16 MiB array that this library holds in device memory
+ * on every GPU that loads it, until the process exits; a call whose
+ * kvarn_decode_workspace_bytes(cfg, num_q_heads) exceeds 16 MiB returns
+ * KVARN_EWORKSPACE.  Nothing is allocated or freed.
+ * The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.  Every
+ * call clears the array's combine tickets on `stream` and then uses the
+ * array, so calls whose work overlaps on the GPU (any two streams, any two
+ * threads) race with each other: order them.  Arguments and results are as
+ * for kvarn_decode_attention.
+ */
+KVARN_API int kvarn_decode_attention_noalloc(const kvarn_config *cfg, const void *q, int num_q_heads,
+                                             float softmax_scale, const kvarn_cache *cache,
+                                             int max_tokens, float *out, void *stream);
+
 /* Static text for a KVARN_* return code. */
 KVARN_API const char *kvarn_strerror(int code);
 

@@ -1,0 +1,42 @@
+"""Decode through the allocation-free entry point (library-held static workspace).
+
+Callers that cannot allocate device memory where they run decode use
+kvarn_decode_attention_noalloc.  It must give the same result as
+kvarn_decode_attention with a caller workspace, call after call, because the
+static array keeps whatever the previous call left in it.  This file is named
+so that pytest collects it last.
+"""
+import numpy as np
+import pytest
+import torch
+
+from bit_kv_cache_token_b200 import kvarn, synth
+
+pytestmark = pytest.mark.gpu
+
+
+def test_noalloc_decode_matches_workspace_decode_twice_in_a_row():
+    S, H, Hq, D, L = 2, 4, 16, 128, 1111
+    cfg = kvarn.Config(S, H, D, max_blocks=10)
+    cache = kvarn.KVCache(cfg)
+    k, v = synth.layer_kv(123, 0, S, H, L, D, device="cuda")
+    kvarn.quantize_blocks(cfg, k, v, cache)
+    for call in range(2):
+        q = synth.queries(200 + call, S, Hq, D, device="cuda")
+        ref = kvarn.decode_attention(cfg, q, cache, max_tokens=L)
+        out = torch.full_like(ref, float("nan"))
+        kvarn.decode_attention_noalloc(cfg, q, cache, L, out)
+        torch.cuda.synchronize()
+        assert int(cache.status.item()) == 0
+        np.testing.assert_allclose(out.cpu().numpy(), ref.cpu().numpy(), rtol=0, atol=2e-3)
+
+
+def test_noalloc_rejects_a_workspace_beyond_the_static_size():
+    cfg = kvarn.Config(8, 8, 128, max_blocks=1)  # 64 (sequence, kv head) pairs, GQA 8: ~17 MB of split partials
+    assert kvarn.decode_workspace_bytes(cfg, 64) > 16 << 20
+    cache = kvarn.KVCache(cfg)
+    q = torch.zeros(8, 64, 128, dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros(q.shape, dtype=torch.float32, device="cuda")
+    with pytest.raises(kvarn.KvarnError) as e:
+        kvarn.decode_attention_noalloc(cfg, q, cache, 0, out)
+    assert e.value.code == kvarn.KVARN_EWORKSPACE
