@@ -74,24 +74,61 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// fp32 pair -> fp16 pairs (hi, lo) with x = hi + lo * 2^-11 to about 2^-22
-// relative.  The remainder is scaled up by 2^11 so that it stays a normal
-// fp16 number whenever hi is; the MMA result of the lo rows is scaled back.
-constexpr float kLoUp = 2048.f;
-constexpr float kLoDown = 1.f / 2048.f;
+// fp32 pair -> fp16 pairs (hi, lo) with x = hi + lo to about 2^-22 relative.
+// (lo may be subnormal: the lo rows of an MMA only need about 11 bits.)
 __device__ __forceinline__ void split_hilo(float x, float y, uint32_t &hi, uint32_t &lo)
 {
     const __half2 h = __floats2half2_rn(x, y);
     const float2 hf = __half22float2(h);
-    const __half2 l = __floats2half2_rn((x - hf.x) * kLoUp, (y - hf.y) * kLoUp);
+    const __half2 l = __floats2half2_rn(x - hf.x, y - hf.y);
     hi = *reinterpret_cast<const uint32_t *>(&h);
     lo = *reinterpret_cast<const uint32_t *>(&l);
 }
 
 // hi rows (c0, c1) plus lo rows (c2, c3) of an accumulator
-__device__ __forceinline__ float2 hilo_sum(const float (&c)[4])
+__device__ __forceinline__ float2 hilo_sum(const float (&c)[4]) { return f2(c[0] + c[2], c[1] + c[3]); }
+
+// Four binary16 values (8 bytes) -> fp32 times `mul`.
+__device__ __forceinline__ float4 h4_to_f4(uint2 w, float mul)
 {
-    return f2(fmaf(c[2], kLoDown, c[0]), fmaf(c[3], kLoDown, c[1]));
+    const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&w.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&w.y));
+    return make_float4(a.x * mul, a.y * mul, b.x * mul, b.y * mul);
+}
+
+// Per-token scales of one record to fp32, one lane per 4 consecutive tokens:
+// out_s[g][t] = s[t][g] * rmul(t) * smul and out_r[t] = r[t]; out_c[d] = c[d] * cmul.
+// rmul(t) is r[t] * tmul when with_r, else 1; tmul is the same for the
+// lane's 4 tokens.
+template <int D, bool WITH_R>
+__device__ __forceinline__ void convert_scales(const unsigned char *rec, float *out_s, float *out_r, float *out_c,
+                                               float smul, float tmul, float cmul)
+{
+    using R = Record<D>;
+    constexpr int NG = D / kGroup;
+    const int lane = threadIdx.x & 31, t0 = 4 * lane;
+    const float4 r4 = h4_to_f4(reinterpret_cast<const uint2 *>(rec + R::kROff)[lane], 1.f);
+    *reinterpret_cast<float4 *>(out_r + t0) = r4;
+    const float rr[4] = {r4.x * tmul, r4.y * tmul, r4.z * tmul, r4.w * tmul};
+    // s of tokens t0..t0+3: 4*NG halves at half index t0*NG (8-byte aligned)
+    const uint2 *sp = reinterpret_cast<const uint2 *>(rec + R::kSOff) + lane * NG;
+    float sv[4 * NG];
+#pragma unroll
+    for (int i = 0; i < NG; ++i) {
+        const float4 f = h4_to_f4(sp[i], smul);
+        sv[4 * i] = f.x; sv[4 * i + 1] = f.y; sv[4 * i + 2] = f.z; sv[4 * i + 3] = f.w;
+    }
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        float4 o;
+        o.x = sv[0 * NG + g] * (WITH_R ? rr[0] : 1.f);
+        o.y = sv[1 * NG + g] * (WITH_R ? rr[1] : 1.f);
+        o.z = sv[2 * NG + g] * (WITH_R ? rr[2] : 1.f);
+        o.w = sv[3 * NG + g] * (WITH_R ? rr[3] : 1.f);
+        *reinterpret_cast<float4 *>(out_s + g * kBlockTokens + t0) = o;
+    }
+    const __half *ch = reinterpret_cast<const __half *>(rec + R::kCOff);
+    for (int d = lane; d < D; d += 32) out_c[d] = __half2float(ch[d]) * cmul;
 }
 
 // The five shifted copies of a code word from which every position is one AND.
@@ -210,8 +247,13 @@ decode_kernel(DecodeArgs a, int hb)
     if (n < 0) n = 0;
     const int nblk = n / kBlockTokens;
     const int ntail = n - nblk * kBlockTokens;
-    const int b0 = split * a.blocks_per_split;
-    const int b1 = min(b0 + a.blocks_per_split, nblk);
+    // split `split` of nsplit covers blocks [split*W/nsplit, (split+1)*W/nsplit) of
+    // W = NB + 2 work slots, NB = max_tokens / T blocks: the last split also
+    // attends the residual tail (about two blocks of work), so it gets fewer blocks
+    const int nbmax = a.max_tokens / kBlockTokens;
+    const long long wslots = nbmax + 2;
+    const int b0 = min((int)(((long long)split * wslots) / a.nsplit), nbmax);
+    const int b1 = min(min((int)(((long long)(split + 1) * wslots) / a.nsplit), nbmax), nblk);
 
     // ---- rotated query of this GQA group, scaled by softmax scale * log2(e)
     const Tin *qg = static_cast<const Tin *>(a.q) + (size_t)unit * GRP * D;
@@ -245,17 +287,7 @@ decode_kernel(DecodeArgs a, int hb)
         float *scr = sm.scr;
 
         // ---- K scales to fp32: sK[g][t] = s * 2^16, rK[t], cK[d]
-        {
-            const __half *sh = reinterpret_cast<const __half *>(krec + R::kSOff);
-            for (int idx = lane; idx < NG * kBlockTokens; idx += 32) {
-                const int t = idx / NG, g = idx % NG;
-                scr[g * kBlockTokens + t] = __half2float(sh[idx]) * kTwo16;
-            }
-            const __half *rh = reinterpret_cast<const __half *>(krec + R::kROff);
-            for (int t = lane; t < kBlockTokens; t += 32) scr[NG * kBlockTokens + t] = __half2float(rh[t]);
-            const __half *ch = reinterpret_cast<const __half *>(krec + R::kCOff);
-            for (int d = lane; d < D; d += 32) scr[(NG + 1) * kBlockTokens + d] = __half2float(ch[d]);
-        }
+        convert_scales<D, false>(krec, scr, scr + NG * kBlockTokens, scr + (NG + 1) * kBlockTokens, kTwo16, 1.f, 1.f);
         __syncwarp();
         const float *sK = scr, *rK = scr + NG * kBlockTokens, *cK = scr + (NG + 1) * kBlockTokens;
 
@@ -307,14 +339,16 @@ decode_kernel(DecodeArgs a, int hb)
             const uint32_t *wp = reinterpret_cast<const uint32_t *>(krec) + (u * 32 + lane) * KW;
 #pragma unroll
             for (int w = 0; w < KW; ++w) kw[w] = CodeWord(wp[w]);
+            // both 8-token n-tiles of the unit at once: independent MMA chains interleave
+            float acc[2][SETS][4];
 #pragma unroll
-            for (int ntl = 0; ntl < 2; ++ntl) {
-                const int nt8 = 2 * u + ntl;
-                float acc[SETS][4];
+            for (int ntl = 0; ntl < 2; ++ntl)
 #pragma unroll
-                for (int st = 0; st < SETS; ++st) acc[st][0] = acc[st][1] = acc[st][2] = acc[st][3] = 0.f;
+                for (int st = 0; st < SETS; ++st) acc[ntl][st][0] = acc[ntl][st][1] = acc[ntl][st][2] = acc[ntl][st][3] = 0.f;
 #pragma unroll
-                for (int kt = 0; kt < NKT; ++kt) {
+            for (int kt = 0; kt < NKT; ++kt) {
+#pragma unroll
+                for (int ntl = 0; ntl < 2; ++ntl) {
                     uint32_t bb[2];
 #pragma unroll
                     for (int cs = 0; cs < 2; ++cs) {
@@ -324,24 +358,35 @@ decode_kernel(DecodeArgs a, int hb)
                         else { word = 2 * F; pos = q - 8 * F + 4 * ntl; }
                         bb[cs] = code_pair(kw[word], pos);
                     }
-                    mma16816(acc[(kt / 2) / C], Aq[kt], bb[0], bb[1]);
+                    mma16816(acc[ntl][(kt / 2) / C], Aq[kt], bb[0], bb[1]);
                 }
-                float accM[4] = {0.f, 0.f, 0.f, 0.f};
-                {
-                    const int t = 8 * nt8 + gl;
-                    const __half *mh = reinterpret_cast<const __half *>(krec + R::kMOff) + t * NG;
+            }
+            float accM[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int ntl = 0; ntl < 2; ++ntl) {
+                const int t = 16 * u + 8 * ntl + gl;
+                const __half *mh = reinterpret_cast<const __half *>(krec + R::kMOff) + t * NG;
+                uint32_t mp = 0u;
+                if constexpr (NG % 2 == 0) {
+                    if (2 * tig < NG) mp = *reinterpret_cast<const uint32_t *>(mh + 2 * tig);
+                } else {
                     const __half m0 = (2 * tig < NG) ? mh[2 * tig] : __float2half(0.f);
                     const __half m1 = (2 * tig + 1 < NG) ? mh[2 * tig + 1] : __float2half(0.f);
-                    __half2 mp = __halves2half2(m0, m1);
-                    mma16816(accM, AM, *reinterpret_cast<uint32_t *>(&mp), 0u);
+                    __half2 m2 = __halves2half2(m0, m1);
+                    mp = *reinterpret_cast<uint32_t *>(&m2);
                 }
+                mma16816(accM[ntl], AM, mp, 0u);
+            }
+#pragma unroll
+            for (int ntl = 0; ntl < 2; ++ntl) {
+                const int nt8 = 2 * u + ntl;
                 const int t0 = 8 * nt8 + 2 * tig;
-                float2 sum = hilo_sum(accM);
+                float2 sum = hilo_sum(accM[ntl]);
 #pragma unroll
                 for (int st = 0; st < SETS; ++st) {
                     const int g = st * C + copy;
                     if (g < NG) {
-                        const float2 P = hilo_sum(acc[st]);
+                        const float2 P = hilo_sum(acc[ntl][st]);
                         const float2 sp = *reinterpret_cast<const float2 *>(sK + g * kBlockTokens + t0);
                         sum = __ffma2_rn(P, sp, sum);
                     }
@@ -377,20 +422,10 @@ decode_kernel(DecodeArgs a, int hb)
             issue_record(&sm.mbar[0], sm.rec[0], kbase + (size_t)(b + 1) * R::kBytes, R::kBytes);
         if (!mbar_wait(&sm.mbar[1], i & 1)) { failed_at = i; break; }
 
-        // ---- V scales: rsV[g][t] = r^V_t s^V_{t,g} e(t), rV[t], cV[d] * 2^16
-        {
-            const __half *sh = reinterpret_cast<const __half *>(vrec + R::kSOff);
-            const __half *rh = reinterpret_cast<const __half *>(vrec + R::kROff);
-            for (int idx = lane; idx < NG * kBlockTokens; idx += 32) {
-                const int t = idx / NG, g = idx % NG;
-                // tokens t with odd t/32 sit at odd code positions (scale 2^-18): times 4
-                const float e = ((t >> 5) & 1) ? 4.f : 1.f;
-                scr[g * kBlockTokens + t] = __half2float(sh[idx]) * __half2float(rh[t]) * e;
-            }
-            for (int t = lane; t < kBlockTokens; t += 32) scr[NG * kBlockTokens + t] = __half2float(rh[t]);
-            const __half *ch = reinterpret_cast<const __half *>(vrec + R::kCOff);
-            for (int d = lane; d < D; d += 32) scr[(NG + 1) * kBlockTokens + d] = __half2float(ch[d]) * kTwo16;
-        }
+        // ---- V scales: rsV[g][t] = r^V_t s^V_{t,g} e(t), rV[t], cV[d] * 2^16, where
+        //      tokens with odd t/32 sit at odd code positions (scale 2^-18): e = 4
+        convert_scales<D, true>(vrec, scr, scr + NG * kBlockTokens, scr + (NG + 1) * kBlockTokens, 1.f,
+                                ((lane >> 3) & 1) ? 4.f : 1.f, kTwo16);
         __syncwarp();
         const float *rsV = scr, *rV = scr + NG * kBlockTokens, *cV = scr + (NG + 1) * kBlockTokens;
 
@@ -448,27 +483,41 @@ decode_kernel(DecodeArgs a, int hb)
             for (int cc = 0; cc < C; ++cc) {
                 const int gg = st * C + cc;
                 if (gg >= NG) continue;
+                // two 8-channel n-tiles at once: independent MMA chains interleave
 #pragma unroll
-                for (int j4 = 0; j4 < kGroup / 8; ++j4) {
-                    const int nt = gg * (kGroup / 8) + j4;
-                    const uint2 vw2 = reinterpret_cast<const uint2 *>(vrec)[nt * 32 + lane];
-                    const CodeWord vw[2] = {CodeWord(vw2.x), CodeWord(vw2.y)};
-                    float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int j4 = 0; j4 < kGroup / 8; j4 += 2) {
+                    const int nt0 = gg * (kGroup / 8) + j4;
+                    CodeWord vw[2][2];
+                    float acc4[2][4];
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const uint2 vw2 = reinterpret_cast<const uint2 *>(vrec)[(nt0 + jj) * 32 + lane];
+                        vw[jj][0] = CodeWord(vw2.x);
+                        vw[jj][1] = CodeWord(vw2.y);
+                        acc4[jj][0] = acc4[jj][1] = acc4[jj][2] = acc4[jj][3] = 0.f;
+                    }
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
-                        uint32_t bb[2];
 #pragma unroll
-                        for (int cs = 0; cs < 2; ++cs) {
-                            const int m = 2 * ks + cs, am = m % 4;
-                            bb[cs] = code_pair(vw[am / 2], 4 * (am % 2) + m / 4);
+                        for (int jj = 0; jj < 2; ++jj) {
+                            uint32_t bb[2];
+#pragma unroll
+                            for (int cs = 0; cs < 2; ++cs) {
+                                const int m = 2 * ks + cs, am = m % 4;
+                                bb[cs] = code_pair(vw[jj][am / 2], 4 * (am % 2) + m / 4);
+                            }
+                            mma16816(acc4[jj], Av[ks], bb[0], bb[1]);
                         }
-                        mma16816(acc4, Av[ks], bb[0], bb[1]);
                     }
                     if (cc == copy) {
-                        const float2 cv = *reinterpret_cast<const float2 *>(cV + 8 * nt + 2 * tig);
-                        const float2 hs = hilo_sum(acc4);
-                        const float2 o = f2(hs.x + bias, hs.y + bias);
-                        orun[nt] = __ffma2_rn(o, cv, orun[nt]);
+#pragma unroll
+                        for (int jj = 0; jj < 2; ++jj) {
+                            const int nt = nt0 + jj;
+                            const float2 cv = *reinterpret_cast<const float2 *>(cV + 8 * nt + 2 * tig);
+                            const float2 hs = hilo_sum(acc4[jj]);
+                            const float2 o = f2(hs.x + bias, hs.y + bias);
+                            orun[nt] = __ffma2_rn(o, cv, orun[nt]);
+                        }
                     }
                 }
             }
@@ -594,34 +643,80 @@ decode_kernel(DecodeArgs a, int hb)
     if (lane == 0) a.tickets[unit] = 0u;
     __threadfence();
 
-    float *obuf = reinterpret_cast<float *>(sm.rec[0]);   // [GRP][D] rotated part
-    float *otl = reinterpret_cast<float *>(sm.rec[1]);    // [GRP][D] tail part
+    float *obuf = reinterpret_cast<float *>(sm.rec[0]);   // [GRP][D] rotated part, then the output
+    float *wbuf = reinterpret_cast<float *>(sm.rec[1]);   // [GRP][slots] log-sum-exp weights, then tail part
+    const int nslot = a.nsplit + 1;                       // block partials and the tail partial
+    // pass 1: per head, lanes over partials: max, weights, normaliser
+    float linv[GRP];
+#pragma unroll
     for (int hh = 0; hh < GRP; ++hh) {
         float M = -INFINITY;
-        for (int i = 0; i <= a.nsplit; ++i) M = fmaxf(M, __ldcg(pbase + ((size_t)i * GRP + hh) * (D + 2)));
+        for (int i = lane; i < nslot; i += 32) M = fmaxf(M, __ldcg(pbase + ((size_t)i * GRP + hh) * (D + 2)));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         float L = 0.f;
-        float orot[D / 32], otail[D / 32];
-#pragma unroll
-        for (int c2 = 0; c2 < D / 32; ++c2) orot[c2] = otail[c2] = 0.f;
-        if (M > -INFINITY) {
-            for (int i = 0; i <= a.nsplit; ++i) {
-                const float *pp = pbase + ((size_t)i * GRP + hh) * (D + 2);
-                const float wgt = exp2f(__ldcg(pp) - M);
-                L = fmaf(__ldcg(pp + 1), wgt, L);
-#pragma unroll
-                for (int c2 = 0; c2 < D / 32; ++c2) {
-                    const float o = __ldcg(pp + 2 + 32 * c2 + lane) * wgt;
-                    if (i < a.nsplit) orot[c2] += o; else otail[c2] += o;
-                }
-            }
+        for (int i = lane; i < nslot; i += 32) {
+            const float *pp = pbase + ((size_t)i * GRP + hh) * (D + 2);
+            const float wgt = M > -INFINITY ? exp2f(__ldcg(pp) - M) : 0.f;
+            L = fmaf(__ldcg(pp + 1), wgt, L);
+            wbuf[hh * (kMaxSplits + 1) + i] = wgt;
         }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        linv[hh] = L > 0.f ? 1.f / L : 0.f;
+    }
+    __syncwarp();
+    // pass 2: lanes over (head, channel); four partials' loads in flight at a time
+    float orot[GRP][D / 32];
+#pragma unroll
+    for (int hh = 0; hh < GRP; ++hh)
+#pragma unroll
+        for (int c2 = 0; c2 < D / 32; ++c2) orot[hh][c2] = 0.f;
+    int i0 = 0;
+    for (; i0 + 4 <= a.nsplit; i0 += 4) {
+        float ov[4][GRP][D / 32];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int hh = 0; hh < GRP; ++hh)
+#pragma unroll
+                for (int c2 = 0; c2 < D / 32; ++c2)
+                    ov[u][hh][c2] = __ldcg(pbase + ((size_t)(i0 + u) * GRP + hh) * (D + 2) + 2 + 32 * c2 + lane);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int hh = 0; hh < GRP; ++hh) {
+                const float wgt = wbuf[hh * (kMaxSplits + 1) + i0 + u];
+#pragma unroll
+                for (int c2 = 0; c2 < D / 32; ++c2) orot[hh][c2] = fmaf(ov[u][hh][c2], wgt, orot[hh][c2]);
+            }
+    }
+    for (; i0 < a.nsplit; ++i0)
+#pragma unroll
+        for (int hh = 0; hh < GRP; ++hh) {
+            const float wgt = wbuf[hh * (kMaxSplits + 1) + i0];
+#pragma unroll
+            for (int c2 = 0; c2 < D / 32; ++c2)
+                orot[hh][c2] = fmaf(__ldcg(pbase + ((size_t)i0 * GRP + hh) * (D + 2) + 2 + 32 * c2 + lane), wgt,
+                                    orot[hh][c2]);
+        }
+    float otail[GRP][D / 32];
+#pragma unroll
+    for (int hh = 0; hh < GRP; ++hh) {
+        const float wgt = wbuf[hh * (kMaxSplits + 1) + a.nsplit];
+#pragma unroll
+        for (int c2 = 0; c2 < D / 32; ++c2)
+            otail[hh][c2] = __ldcg(pbase + ((size_t)a.nsplit * GRP + hh) * (D + 2) + 2 + 32 * c2 + lane) * wgt;
+    }
+    __syncwarp();  // wbuf is read: the tail part may now reuse it
+    float *otl = wbuf;
+#pragma unroll
+    for (int hh = 0; hh < GRP; ++hh)
 #pragma unroll
         for (int c2 = 0; c2 < D / 32; ++c2) {
-            obuf[hh * D + 32 * c2 + lane] = orot[c2] * inv;
-            otl[hh * D + 32 * c2 + lane] = otail[c2] * inv;
+            obuf[hh * D + 32 * c2 + lane] = orot[hh][c2] * linv[hh];
+            otl[hh * D + 32 * c2 + lane] = otail[hh][c2] * linv[hh];
         }
-    }
     __syncwarp();
     warp_fwht<D>(obuf, GRP, hb);
     float *out = a.out + (size_t)unit * GRP * D;

@@ -163,14 +163,12 @@ int kvarn_decode_attention(const kvarn_config *cfg, const void *q, int num_q_hea
     // are resident at once (one CTA of decode_warps_per_cta warps per SM)
     const int units = cfg->num_seqs * cfg->num_kv_heads;
     const int nblk = max_tokens / cfg->block_tokens;
-    int nsplit = 1, bps = nblk > 0 ? nblk : 1;
+    int nsplit = 1;
     if (nblk > 0) {
         int ns = num_sms() * decode_warps_per_cta(cfg->head_dim, grp) / units;
         ns = ns < 1 ? 1 : ns;
         ns = ns > nblk ? nblk : ns;
-        ns = ns > kMaxSplits ? kMaxSplits : ns;
-        bps = (nblk + ns - 1) / ns;
-        nsplit = (nblk + bps - 1) / bps;
+        nsplit = ns > kMaxSplits ? kMaxSplits : ns;
     }
     DecodeArgs a;
     a.q = q;
@@ -183,7 +181,7 @@ int kvarn_decode_attention(const kvarn_config *cfg, const void *q, int num_q_hea
     const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)cfg->head_dim);
     a.scale_log2 = scale * 1.4426950408889634f;
     a.num_kv_heads = cfg->num_kv_heads; a.grp = grp; a.max_blocks = cfg->max_blocks;
-    a.max_tokens = max_tokens; a.num_units = units; a.nsplit = nsplit; a.blocks_per_split = bps;
+    a.max_tokens = max_tokens; a.num_units = units; a.nsplit = nsplit;
     return cuda_status(run_decode(*cfg, a, static_cast<cudaStream_t>(stream)));
 }
 

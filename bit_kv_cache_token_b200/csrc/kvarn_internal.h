@@ -47,7 +47,7 @@ struct DecodeArgs {
     float scale_log2;           // softmax scale * log2(e)
     int num_kv_heads, grp, max_blocks, max_tokens;
     int num_units;              // S * Hkv
-    int nsplit, blocks_per_split;  // warps per unit, blocks per warp
+    int nsplit;                 // warps per unit; each takes a contiguous range of blocks
 };
 
 cudaError_t run_quantize(const kvarn_config &c, const QuantArgs &a, cudaStream_t st);
