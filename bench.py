@@ -109,42 +109,30 @@ class ClockSampler:
 
 
 def _dist_setup(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
+    from bit_kv_cache_token_b200 import dp
+    world, rank, local = dp.world_from_env()
+    torch.cuda.set_device(local if world > 1 else 0)
+    dp.init(world, "nccl", torch.device("cuda", local))
     return world, rank, local
 
 
 def _barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    from bit_kv_cache_token_b200 import dp
+    dp.barrier(world)
 
 
 def _max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from bit_kv_cache_token_b200 import dp
+    return dp.max_over_ranks(x, world, "cuda")
 
 
-# --------------------------------------------------------------------------------- GPU arm
 def run_kvarn(args, world, rank, local):
     from bit_kv_cache_token_b200 import kvarn, synth
 
     dev = torch.device("cuda", local)
     cfg = kvarn.Config(S, HKV, D, max_blocks=32768 // T_BLK, hadamard=D, sweeps=4, dtype=kvarn.KVARN_BF16)
-    seed = 2 + 1000 * rank
+    from bit_kv_cache_token_b200 import dp
+    seed = dp.rank_seed(2, rank)
     # ---- caches: 36 layers prefilled to CTX0 tokens through the bulk quantiser
     caches = []
     for layer in range(LAYERS):
@@ -219,8 +207,7 @@ def run_kvarn(args, world, rank, local):
         dec_ms.append(a.elapsed_time(b))  # last replay's probe launches
     ms_total = _max_over_ranks(t0.elapsed_time(t1), world)
     ms_step = ms_total / args.steps
-    tokens = S * T_BLK * args.steps * world
-    value = tokens / (ms_total / 1e3)
+    value = dp.aggregate_rate(S * T_BLK * args.steps, ms_total / 1e3, world)
 
     # decode-only roofline: events around each layer's decode at sub-step probe_j (context CTX0+probe_j+1)
     dec_avg_ms = statistics.mean(dec_ms)
@@ -248,7 +235,7 @@ def run_kvarn(args, world, rank, local):
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = tokens / (e2e_ms / 1e3)
+    e2e_value = dp.aggregate_rate(S * T_BLK * args.steps, e2e_ms / 1e3, world)
     h2d = (qs.numel() + ks.numel() + vs.numel()) * 2
     d2h = outs.numel() * 4
     del graph
@@ -466,9 +453,8 @@ def main():
         if cpu:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    from bit_kv_cache_token_b200 import dp
+    dp.finish(world)
 
 
 if __name__ == "__main__":

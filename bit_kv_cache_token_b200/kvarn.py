@@ -24,6 +24,7 @@ KVARN_ECUDA = -4
 KVARN_STATUS_CAPACITY = 1
 KVARN_STATUS_NONFINITE = 2
 KVARN_STATUS_LENGTH = 4
+KVARN_STATUS_TIMEOUT = 8
 KVARN_F32 = 0
 KVARN_BF16 = 1
 
