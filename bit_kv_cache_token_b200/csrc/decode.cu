@@ -13,13 +13,18 @@
 // query; the combine merges all partials with log-sum-exp weights, rotates
 // the block part back and adds the tail part.
 //
-// B200 mapping.  One warp streams a contiguous range of 128-token blocks of
-// one (sequence, kv head) with its own online softmax; the records reach
-// shared memory by cp.async.bulk (TMA), one buffer each for K and V guarded
-// by mbarriers: the next K record is requested as soon as the scores are
-// done, the next V record as soon as P V is done, so each copy overlaps half
-// a block of this warp's work and the whole work of the SM's other warps.  Both contractions run on tensor cores (mma.sync m16n8k16, fp16
-// in, fp32 accumulate):
+// B200 mapping.  The work of a launch is a list of items, unit by unit (a
+// unit is one (sequence, kv head)): the unit's max_tokens / 128 blocks, then
+// one item for its residual tail.  Every warp of a persistent grid (one CTA
+// per SM) takes an equal contiguous range of that list, so the load is even
+// whatever the number of units and their lengths relative to the SM count.
+// Where a range crosses into a new unit the warp starts a new online softmax.
+// The records reach shared memory by cp.async.bulk (TMA), one buffer each
+// for K and V guarded by mbarriers: the next K record is requested as soon
+// as the scores are done, the next V record as soon as P V is done, so each
+// copy overlaps half a block of this warp's work and the whole work of the
+// SM's other warps.  Both contractions run on tensor cores (mma.sync
+// m16n8k16, fp16 in, fp32 accumulate):
 //   scores: A = q' (rows: query heads; hi/lo fp16 split in rows 0-7 / 8-15),
 //           B = K codes (k = channels, n = 8 tokens);
 //   P V:    A = p r s (rows: heads, hi/lo), B = V codes (k = tokens, n = 8 channels).
@@ -31,8 +36,15 @@
 // (it depends only on the contracted index), the remaining 2^-16 into the
 // scales.  When the GQA group has fewer than 8 heads, the spare rows
 // carry copies of the heads working on other channel groups, so every lane
-// does useful work.  The last warp of a (sequence, kv head) to finish,
-// found with an atomic ticket, combines; no warp ever waits for another.
+// does useful work.  The tail item is attended on CUDA cores with
+// load-parallel loops.
+//
+// Merging.  Every (warp, unit) segment writes one partial (m, l, o_rot per
+// head); the tail item writes the unit's tail partial.  A per-unit ticket
+// counts the items whose partials are written; the warp that completes it
+// merges the unit itself when few warps covered it, and otherwise marks the
+// unit for its CTA, whose warps merge it together after they have all
+// finished their ranges.  No warp ever waits for another CTA.
 #include <math.h>
 
 #include "kvarn_common.cuh"
@@ -215,9 +227,35 @@ __device__ void warp_fwht(float *x, int nvec, int hb)
     __syncwarp();
 }
 
+
+// ---- the partition of the item list over the warps of the grid -----------
+// warp w takes items [w * total / nw, (w + 1) * total / nw)
+__device__ __forceinline__ long long part_begin(long long w, long long total, long long nw)
+{
+    return w * total / nw;
+}
+
+// the warp whose range holds item i
+__device__ __forceinline__ long long part_owner(long long i, long long total, long long nw)
+{
+    return ((i + 1) * nw + total - 1) / total - 1;
+}
+
+// Slot layout of a partial: per head [m, l, pad, pad, o[D]] (16-byte aligned rows).
+template <int D>
+__host__ __device__ constexpr int slot_row() { return D + 4; }
+
+// Partials are merged by the completing warp alone up to this many warps per unit.
+constexpr int kWarpMergeMax = 8;
+// Marker of a unit whose merge the completing warp left to its CTA.
+constexpr uint32_t kMergeFlag = 0x80000000u;
+
+// Blocks [b0, b1) of one unit into the running (m_run, l_run, orun).
+// Returns false if a staged copy did not arrive in time (after letting the
+// copies still in flight land, bounded); the warp then stops using TMA.
 template <int D, int GRP, typename Tin>
-__global__ void __launch_bounds__(dec_warps<D, GRP>() * 32, 1)
-decode_kernel(DecodeArgs a, int hb)
+__device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, const unsigned char *vbase, int b0,
+                           int b1, uint32_t &kph, uint32_t &vph, float &m_run, float &l_run, float2 (&orun)[D / 8])
 {
     using R = Record<D>;
     constexpr int NG = D / kGroup;          // channel groups
@@ -227,61 +265,23 @@ decode_kernel(DecodeArgs a, int hb)
     constexpr int SETS = (NG + C - 1) / C;  // groups handled per copy
     constexpr int KW = D / 32;              // K code words per (16-token unit, lane)
     constexpr int F = D / 64;
-
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    DecWarpSmem<D, GRP> &sm = reinterpret_cast<DecWarpSmem<D, GRP> *>(smem_raw)[warp];
-    const int item = blockIdx.x * dec_warps<D, GRP>() + warp;
-    const int nitems = a.num_units * a.nsplit;
-    if (item >= nitems) return;
-    const int unit = item / a.nsplit, split = item % a.nsplit;
-    const int s = unit / a.num_kv_heads;
+    const int lane = threadIdx.x & 31;
     const int gl = lane >> 2, tig = lane & 3;  // mma groupID, thread in group
     const int copy = gl / GRP, h = gl % GRP;
 
-    int n = a.n_tokens[s];
-    if (n > a.max_tokens) {
-        if (lane == 0 && split == 0) status_or(a.status, KVARN_STATUS_LENGTH);
-        n = a.max_tokens;
-    }
-    if (n < 0) n = 0;
-    const int nblk = n / kBlockTokens;
-    const int ntail = n - nblk * kBlockTokens;
-    // split `split` of nsplit covers blocks [split*W/nsplit, (split+1)*W/nsplit) of
-    // W = NB + 2 work slots, NB = max_tokens / T blocks: the last split also
-    // attends the residual tail (about two blocks of work), so it gets fewer blocks
-    const int nbmax = a.max_tokens / kBlockTokens;
-    const long long wslots = nbmax + 2;
-    const int b0 = min((int)(((long long)split * wslots) / a.nsplit), nbmax);
-    const int b1 = min(min((int)(((long long)(split + 1) * wslots) / a.nsplit), nbmax), nblk);
-
-    // ---- rotated query of this GQA group, scaled by softmax scale * log2(e)
-    const Tin *qg = static_cast<const Tin *>(a.q) + (size_t)unit * GRP * D;
-    for (int i = lane; i < GRP * D; i += 32) (&sm.qbuf[0][0])[i] = In<Tin>::load1(qg + i) * a.scale_log2;
-    __syncwarp();
-    warp_fwht<D>(&sm.qbuf[0][0], GRP, hb);
-
-    float m_run = -INFINITY, l_run = 0.f;
-    float2 orun[NNT];
-#pragma unroll
-    for (int i = 0; i < NNT; ++i) orun[i] = f2(0.f, 0.f);
-    int failed_at = -1;  // block index whose copy did not arrive in time
-
-    const unsigned char *kbase = static_cast<const unsigned char *>(a.k_records) + (size_t)unit * a.max_blocks * R::kBytes;
-    const unsigned char *vbase = static_cast<const unsigned char *>(a.v_records) + (size_t)unit * a.max_blocks * R::kBytes;
+    if (b0 >= b1) return true;
     if (lane == 0) {
-        mbar_init(&sm.mbar[0]);
-        mbar_init(&sm.mbar[1]);
-    }
-    __syncwarp();
-    if (lane == 0 && b0 < b1) {
         issue_record(&sm.mbar[0], sm.rec[0], kbase + (size_t)b0 * R::kBytes, R::kBytes);
         issue_record(&sm.mbar[1], sm.rec[1], vbase + (size_t)b0 * R::kBytes, R::kBytes);
     }
-
     for (int b = b0; b < b1; ++b) {
-        const int i = b - b0;
-        if (!mbar_wait(&sm.mbar[0], i & 1)) { failed_at = i; break; }
+        if (!mbar_wait(&sm.mbar[0], kph)) {
+            // in flight: K and V of block b
+            if (lane == 0) { mbar_wait(&sm.mbar[0], kph); mbar_wait(&sm.mbar[1], vph); }
+            __syncwarp();
+            return false;
+        }
+        kph ^= 1u;
         const unsigned char *krec = sm.rec[0];
         const unsigned char *vrec = sm.rec[1];
         float *scr = sm.scr;
@@ -420,7 +420,16 @@ decode_kernel(DecodeArgs a, int hb)
         __syncwarp();  // every lane is done with the K record and the K scales
         if (lane == 0 && b + 1 < b1)
             issue_record(&sm.mbar[0], sm.rec[0], kbase + (size_t)(b + 1) * R::kBytes, R::kBytes);
-        if (!mbar_wait(&sm.mbar[1], i & 1)) { failed_at = i; break; }
+        if (!mbar_wait(&sm.mbar[1], vph)) {
+            // in flight: V of block b and K of block b + 1
+            if (lane == 0) {
+                mbar_wait(&sm.mbar[1], vph);
+                if (b + 1 < b1) mbar_wait(&sm.mbar[0], kph);
+            }
+            __syncwarp();
+            return false;
+        }
+        vph ^= 1u;
 
         // ---- V scales: rsV[g][t] = r^V_t s^V_{t,g} e(t), rV[t], cV[d] * 2^16, where
         //      tokens with odd t/32 sit at odd code positions (scale 2^-18): e = 4
@@ -528,239 +537,481 @@ decode_kernel(DecodeArgs a, int hb)
         if (lane == 0 && b + 1 < b1)
             issue_record(&sm.mbar[1], sm.rec[1], vbase + (size_t)(b + 1) * R::kBytes, R::kBytes);
     }
-    if (failed_at >= 0) {
-        // let the copies this warp may still have in flight land (bounded), then report
-        if (lane == 0) {
-            // at most one copy per buffer can be outstanding: the one of block failed_at
-            // (or of failed_at + 1 for K when the V wait gave up)
-            mbar_wait(&sm.mbar[0], failed_at & 1);
-            if (failed_at + 1 < b1 - b0) mbar_wait(&sm.mbar[0], (failed_at + 1) & 1);
-            mbar_wait(&sm.mbar[1], failed_at & 1);
-            status_or(a.status, KVARN_STATUS_TIMEOUT);
-        }
-        __syncwarp();
-        m_run = -INFINITY;
-        l_run = 0.f;
-#pragma unroll
-        for (int i2 = 0; i2 < NNT; ++i2) orun[i2] = f2(0.f, 0.f);
-    }
+    return true;
+}
 
-    // ---- this warp's block partial: (m, l, o_rot) per head
-    const int slots = kMaxSplits + 1;
-    float *pbase = a.partials + (size_t)unit * slots * GRP * (D + 2);
-    {
-        float *pp = pbase + ((size_t)split * GRP + h) * (D + 2);
-        float lsum = l_run;
-        lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
-        lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
-        if (copy == 0 && tig == 0) { pp[0] = m_run; pp[1] = lsum; }
-#pragma unroll
-        for (int nt = 0; nt < NNT; ++nt) {
-            if ((nt / (kGroup / 8)) % C == copy)
-                *reinterpret_cast<float2 *>(pp + 2 + 8 * nt + 2 * tig) = orun[nt];
-        }
+// The residual tail of one unit: unrotated query, CUDA cores.  Writes the
+// tail partial (m, l, o per head, unrotated basis) to dst.
+template <int D, int GRP, typename Tin>
+__device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int unit, int ntail, float *dst)
+{
+    constexpr int QC = D / 4;   // channels per quarter of a row
+    constexpr int QP = QC + 4;  // padded quarter stride: the four quarters sit in different banks
+    constexpr int SR = slot_row<D>();
+    const int lane = threadIdx.x & 31;
+    float *ps = reinterpret_cast<float *>(sm.rec[0]);  // [128][GRP] scores, then weights
+    float *qt = ps + kBlockTokens * GRP;               // [GRP][4][QP] query, scaled
+    static_assert(sizeof(float) * (kBlockTokens * GRP + GRP * 4 * QP) <= sizeof(sm.rec), "tail scratch");
+    const Tin *qg = static_cast<const Tin *>(a.q) + (size_t)unit * GRP * D;
+    for (int i = lane; i < GRP * D; i += 32) {
+        const int hh = i / D, d = i % D;
+        qt[(hh * 4 + d / QC) * QP + d % QC] = In<Tin>::load1(qg + i) * a.scale_log2;
     }
-
-    // ---- residual tail (last split only): unrotated query, lanes over tokens
-    if (split == a.nsplit - 1) {
-        float *pt = pbase + (size_t)a.nsplit * GRP * (D + 2);  // tail slot
-        for (int i = lane; i < GRP * D; i += 32) (&sm.qbuf[0][0])[i] = In<Tin>::load1(qg + i) * a.scale_log2;
-        __syncwarp();
-        const Tin *kt = static_cast<const Tin *>(a.k_tail) + (size_t)unit * kBlockTokens * D;
-        const Tin *vt = static_cast<const Tin *>(a.v_tail) + (size_t)unit * kBlockTokens * D;
-        float st[4][GRP];
+    __syncwarp();
+    // scores: 8 tokens at a time, lane = (token, quarter); the quarters are summed by shuffles
+    const Tin *kt = static_cast<const Tin *>(a.k_tail) + (size_t)unit * kBlockTokens * D;
+    const int tt = lane >> 2, qq = lane & 3;
+    for (int t0 = 0; t0 < ntail; t0 += 8) {
+        const int t = t0 + tt;
+        float acc[GRP];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int t = lane + 32 * i;
+        for (int hh = 0; hh < GRP; ++hh) acc[hh] = 0.f;
+        if (t < ntail) {
+            float kv[QC];
 #pragma unroll
-            for (int hh = 0; hh < GRP; ++hh) st[i][hh] = -INFINITY;
-            if (t < ntail) {
+            for (int c8 = 0; c8 < QC; c8 += 8) {
+                float k8[8];
+                In<Tin>::load8(kt + (size_t)t * D + qq * QC + c8, k8);
 #pragma unroll
-                for (int hh = 0; hh < GRP; ++hh) st[i][hh] = 0.f;
-                for (int d = 0; d < D; d += 8) {
-                    float kv[8];
-                    In<Tin>::load8(kt + (size_t)t * D + d, kv);
+                for (int e = 0; e < 8; ++e) kv[c8 + e] = k8[e];
+            }
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
+            for (int hh = 0; hh < GRP; ++hh) {
+                const float *qr = qt + (hh * 4 + qq) * QP;
 #pragma unroll
-                        for (int hh = 0; hh < GRP; ++hh) st[i][hh] = fmaf(sm.qbuf[hh][d + e], kv[e], st[i][hh]);
+                for (int c4 = 0; c4 < QC; c4 += 4) {
+                    const float4 qv = *reinterpret_cast<const float4 *>(qr + c4);
+                    acc[hh] = fmaf(qv.x, kv[c4], acc[hh]);
+                    acc[hh] = fmaf(qv.y, kv[c4 + 1], acc[hh]);
+                    acc[hh] = fmaf(qv.z, kv[c4 + 2], acc[hh]);
+                    acc[hh] = fmaf(qv.w, kv[c4 + 3], acc[hh]);
                 }
             }
         }
-        float mt[GRP], lt[GRP];
 #pragma unroll
         for (int hh = 0; hh < GRP; ++hh) {
-            float mx = fmaxf(fmaxf(st[0][hh], st[1][hh]), fmaxf(st[2][hh], st[3][hh]));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            mt[hh] = mx;
-            float ssum = 0.f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                st[i][hh] = (lane + 32 * i < ntail) ? exp2f(st[i][hh] - mx) : 0.f;
-                ssum += st[i][hh];
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
-            lt[hh] = ssum;
+            acc[hh] += __shfl_xor_sync(0xffffffffu, acc[hh], 1);
+            acc[hh] += __shfl_xor_sync(0xffffffffu, acc[hh], 2);
         }
-        float ot[GRP][D / 32];
+        if (qq == 0 && t < ntail) {
 #pragma unroll
-        for (int hh = 0; hh < GRP; ++hh)
-#pragma unroll
-            for (int c2 = 0; c2 < D / 32; ++c2) ot[hh][c2] = 0.f;
-        for (int t = 0; t < ntail; ++t) {
-            float pv[GRP];
-#pragma unroll
-            for (int hh = 0; hh < GRP; ++hh) {
-                const float v0 = st[0][hh], v1 = st[1][hh], v2 = st[2][hh], v3 = st[3][hh];
-                const float mine = (t >> 5) == 0 ? v0 : (t >> 5) == 1 ? v1 : (t >> 5) == 2 ? v2 : v3;
-                pv[hh] = __shfl_sync(0xffffffffu, mine, t & 31);
-            }
-#pragma unroll
-            for (int c2 = 0; c2 < D / 32; ++c2) {
-                const float vv = In<Tin>::load1(vt + (size_t)t * D + 32 * c2 + lane);
-#pragma unroll
-                for (int hh = 0; hh < GRP; ++hh) ot[hh][c2] = fmaf(pv[hh], vv, ot[hh][c2]);
-            }
-        }
-#pragma unroll
-        for (int hh = 0; hh < GRP; ++hh) {
-            float *pp = pt + (size_t)hh * (D + 2);
-            if (lane == 0) { pp[0] = ntail > 0 ? mt[hh] : -INFINITY; pp[1] = lt[hh]; }
-#pragma unroll
-            for (int c2 = 0; c2 < D / 32; ++c2) pp[2 + 32 * c2 + lane] = ot[hh][c2];
+            for (int hh = 0; hh < GRP; ++hh) ps[t * GRP + hh] = acc[hh];
         }
     }
-
-    // ---- arrival ticket; the last warp of this (sequence, kv head) combines
     __syncwarp();
-    __threadfence();
-    unsigned prev = 0;
-    if (lane == 0) prev = atomicAdd(a.tickets + unit, 1u);
-    prev = __shfl_sync(0xffffffffu, prev, 0);
-    if (prev != (unsigned)a.nsplit - 1u) return;
-    if (lane == 0) a.tickets[unit] = 0u;
-    __threadfence();
-
-    float *obuf = reinterpret_cast<float *>(sm.rec[0]);   // [GRP][D] rotated part, then the output
-    float *wbuf = reinterpret_cast<float *>(sm.rec[1]);   // [GRP][slots] log-sum-exp weights, then tail part
-    const int nslot = a.nsplit + 1;                       // block partials and the tail partial
-    // pass 1: per head, lanes over partials: max, weights, normaliser
-    float linv[GRP];
+    // softmax over the tail tokens, lanes over tokens
+    float mt[GRP], lt[GRP];
 #pragma unroll
     for (int hh = 0; hh < GRP; ++hh) {
+        float sv[4], mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int t = lane + 32 * j;
+            sv[j] = t < ntail ? ps[t * GRP + hh] : -INFINITY;
+            mx = fmaxf(mx, sv[j]);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int t = lane + 32 * j;
+            const float p = t < ntail ? exp2f(sv[j] - mx) : 0.f;
+            if (t < ntail) ps[t * GRP + hh] = p;
+            sum += p;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        mt[hh] = ntail > 0 ? mx : -INFINITY;
+        lt[hh] = sum;
+    }
+    __syncwarp();
+    // P V: lanes over channel quads, eight tokens' loads in flight
+    const Tin *vt = static_cast<const Tin *>(a.v_tail) + (size_t)unit * kBlockTokens * D;
+    const int c0 = 4 * lane;
+    const bool act = c0 < D;
+    float4 o[GRP];
+#pragma unroll
+    for (int hh = 0; hh < GRP; ++hh) o[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int t0 = 0; t0 < ntail; t0 += 8) {
+        float4 vv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            vv[u] = (act && t0 + u < ntail) ? In<Tin>::load4(vt + (size_t)(t0 + u) * D + c0)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (t0 + u >= ntail) break;
+#pragma unroll
+            for (int hh = 0; hh < GRP; ++hh) {
+                const float p = ps[(t0 + u) * GRP + hh];
+                o[hh].x = fmaf(p, vv[u].x, o[hh].x);
+                o[hh].y = fmaf(p, vv[u].y, o[hh].y);
+                o[hh].z = fmaf(p, vv[u].z, o[hh].z);
+                o[hh].w = fmaf(p, vv[u].w, o[hh].w);
+            }
+        }
+    }
+#pragma unroll
+    for (int hh = 0; hh < GRP; ++hh) {
+        float *row = dst + hh * SR;
+        if (lane == 0) { row[0] = mt[hh]; row[1] = lt[hh]; }
+        if (act) *reinterpret_cast<float4 *>(row + 4 + c0) = o[hh];
+    }
+    __syncwarp();
+}
+
+// Merge of one unit by a single warp (few partials): block partials from the
+// slots of warps [wf, wl] (empty ranges skipped), the tail partial, the
+// un-rotation, the output.  Uses the warp's record buffers as scratch.
+template <int D, int GRP>
+__device__ void warp_merge(const DecodeArgs &a, int hb, DecWarpSmem<D, GRP> &sm, int unit, long long wf, long long wl,
+                           long long total, long long nw)
+{
+    constexpr int SR = slot_row<D>();
+    const int lane = threadIdx.x & 31;
+    const float *tl = a.tail_partials + (size_t)unit * GRP * SR;
+    float *obuf = reinterpret_cast<float *>(sm.rec[0]);  // [GRP][D]
+    float *otl = reinterpret_cast<float *>(sm.rec[1]);   // [GRP][D]
+    const int P = (int)(wl - wf + 1);
+    for (int hh = 0; hh < GRP; ++hh) {
+        // lanes over partials: the maximum, then weights and the normaliser
         float M = -INFINITY;
-        for (int i = lane; i < nslot; i += 32) M = fmaxf(M, __ldcg(pbase + ((size_t)i * GRP + hh) * (D + 2)));
+        for (int p = lane; p < P; p += 32) {
+            const long long w = wf + p;
+            if (part_begin(w, total, nw) < part_begin(w + 1, total, nw))
+                M = fmaxf(M, __ldcg(a.partials + (size_t)(w + unit) * GRP * SR + hh * SR));
+        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float mtl = __ldcg(tl + hh * SR);
+        M = fmaxf(M, mtl);
         float L = 0.f;
-        for (int i = lane; i < nslot; i += 32) {
-            const float *pp = pbase + ((size_t)i * GRP + hh) * (D + 2);
-            const float wgt = M > -INFINITY ? exp2f(__ldcg(pp) - M) : 0.f;
-            L = fmaf(__ldcg(pp + 1), wgt, L);
-            wbuf[hh * (kMaxSplits + 1) + i] = wgt;
+        float acc[D / 32];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) acc[c] = 0.f;
+        for (int p = 0; p < P; ++p) {
+            const long long w = wf + p;
+            if (!(part_begin(w, total, nw) < part_begin(w + 1, total, nw))) continue;
+            const float *row = a.partials + (size_t)(w + unit) * GRP * SR + hh * SR;
+            const float m = __ldcg(row);
+            const float wgt = M > -INFINITY ? exp2f(m - M) : 0.f;
+            if (wgt == 0.f) continue;
+            L = fmaf(__ldcg(row + 1), wgt, L);
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) acc[c] = fmaf(__ldcg(row + 4 + 32 * c + lane), wgt, acc[c]);
         }
+        const float wt = M > -INFINITY ? exp2f(mtl - M) : 0.f;
+        L = fmaf(__ldcg(tl + hh * SR + 1), wt, L);
+        const float linv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-        linv[hh] = L > 0.f ? 1.f / L : 0.f;
-    }
-    __syncwarp();
-    // pass 2: lanes over (head, channel); four partials' loads in flight at a time
-    float orot[GRP][D / 32];
-#pragma unroll
-    for (int hh = 0; hh < GRP; ++hh)
-#pragma unroll
-        for (int c2 = 0; c2 < D / 32; ++c2) orot[hh][c2] = 0.f;
-    int i0 = 0;
-    for (; i0 + 4 <= a.nsplit; i0 += 4) {
-        float ov[4][GRP][D / 32];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-            for (int hh = 0; hh < GRP; ++hh)
-#pragma unroll
-                for (int c2 = 0; c2 < D / 32; ++c2)
-                    ov[u][hh][c2] = __ldcg(pbase + ((size_t)(i0 + u) * GRP + hh) * (D + 2) + 2 + 32 * c2 + lane);
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-            for (int hh = 0; hh < GRP; ++hh) {
-                const float wgt = wbuf[hh * (kMaxSplits + 1) + i0 + u];
-#pragma unroll
-                for (int c2 = 0; c2 < D / 32; ++c2) orot[hh][c2] = fmaf(ov[u][hh][c2], wgt, orot[hh][c2]);
-            }
-    }
-    for (; i0 < a.nsplit; ++i0)
-#pragma unroll
-        for (int hh = 0; hh < GRP; ++hh) {
-            const float wgt = wbuf[hh * (kMaxSplits + 1) + i0];
-#pragma unroll
-            for (int c2 = 0; c2 < D / 32; ++c2)
-                orot[hh][c2] = fmaf(__ldcg(pbase + ((size_t)i0 * GRP + hh) * (D + 2) + 2 + 32 * c2 + lane), wgt,
-                                    orot[hh][c2]);
+        for (int c = 0; c < D / 32; ++c) {
+            obuf[hh * D + 32 * c + lane] = acc[c] * linv;
+            otl[hh * D + 32 * c + lane] = wt > 0.f ? __ldcg(tl + hh * SR + 4 + 32 * c + lane) * wt * linv : 0.f;
         }
-    float otail[GRP][D / 32];
-#pragma unroll
-    for (int hh = 0; hh < GRP; ++hh) {
-        const float wgt = wbuf[hh * (kMaxSplits + 1) + a.nsplit];
-#pragma unroll
-        for (int c2 = 0; c2 < D / 32; ++c2)
-            otail[hh][c2] = __ldcg(pbase + ((size_t)a.nsplit * GRP + hh) * (D + 2) + 2 + 32 * c2 + lane) * wgt;
     }
-    __syncwarp();  // wbuf is read: the tail part may now reuse it
-    float *otl = wbuf;
-#pragma unroll
-    for (int hh = 0; hh < GRP; ++hh)
-#pragma unroll
-        for (int c2 = 0; c2 < D / 32; ++c2) {
-            obuf[hh * D + 32 * c2 + lane] = orot[hh][c2] * linv[hh];
-            otl[hh * D + 32 * c2 + lane] = otail[hh][c2] * linv[hh];
-        }
     __syncwarp();
     warp_fwht<D>(obuf, GRP, hb);
     float *out = a.out + (size_t)unit * GRP * D;
     for (int i = lane; i < GRP * D; i += 32) out[i] = obuf[i] + otl[i];
+    __syncwarp();
+}
+
+// Merge of one unit by all warps of the CTA (many partials).  Every thread
+// of the CTA calls it with the same arguments; the whole dynamic shared
+// memory is scratch.
+template <int D, int GRP>
+__device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int unit, long long wf, long long wl,
+                          long long total, long long nw)
+{
+    constexpr int W = dec_warps<D, GRP>();
+    constexpr int NT = W * 32;
+    constexpr int SR = slot_row<D>();
+    constexpr int NQ = GRP * D / 4;  // float4 columns of a unit's output
+    constexpr int G = NT / NQ;       // partial groups summed in parallel
+    static_assert(G >= 1, "merge layout");
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int P = (int)(wl - wf + 1);
+    const float *tl = a.tail_partials + (size_t)unit * GRP * SR;
+
+    // scratch, every array starting on a 16-byte boundary
+    constexpr int SMALL = (W * GRP + 3 * GRP + 3) & ~3;      // red [W][GRP], Mh, Lh, Wt [GRP]
+    float4 *acc4 = reinterpret_cast<float4 *>(smem);         // [G][NQ]
+    float *obuf = reinterpret_cast<float *>(acc4 + G * NQ);  // [GRP][D]
+    float *otl = obuf + GRP * D;                             // [GRP][D]
+    float *red = otl + GRP * D;
+    float *Mh = red + W * GRP;
+    float *Lh = Mh + GRP;
+    float *Wt = Lh + GRP;
+    float *wts = red + SMALL;                                // [P][GRP]
+
+    const int hh = tid % GRP;  // NT is a multiple of 32, so every thread keeps one head
+    float mx = -INFINITY;
+    for (int idx = tid; idx < P * GRP; idx += NT) {
+        const long long w = wf + idx / GRP;
+        if (part_begin(w, total, nw) < part_begin(w + 1, total, nw))
+            mx = fmaxf(mx, __ldcg(a.partials + (size_t)(w + unit) * GRP * SR + hh * SR));
+    }
+    for (int o = GRP; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane < GRP) red[warp * GRP + lane] = mx;
+    __syncthreads();
+    if (tid < GRP) {
+        float M = __ldcg(tl + tid * SR);
+        for (int w = 0; w < W; ++w) M = fmaxf(M, red[w * GRP + tid]);
+        Mh[tid] = M;
+    }
+    __syncthreads();
+    const float M = Mh[hh];
+    float ls = 0.f;
+    for (int idx = tid; idx < P * GRP; idx += NT) {
+        const long long w = wf + idx / GRP;
+        float wgt = 0.f;
+        if (M > -INFINITY && part_begin(w, total, nw) < part_begin(w + 1, total, nw)) {
+            const float *row = a.partials + (size_t)(w + unit) * GRP * SR + hh * SR;
+            wgt = exp2f(__ldcg(row) - M);
+            ls = fmaf(__ldcg(row + 1), wgt, ls);
+        }
+        wts[idx] = wgt;
+    }
+    for (int o = GRP; o < 32; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+    __syncthreads();  // every thread has read red
+    if (lane < GRP) red[warp * GRP + lane] = ls;
+    __syncthreads();
+    if (tid < GRP) {
+        const float Mt = Mh[tid];
+        const float wt = Mt > -INFINITY ? exp2f(__ldcg(tl + tid * SR) - Mt) : 0.f;
+        float L = wt * __ldcg(tl + tid * SR + 1);
+        for (int w = 0; w < W; ++w) L += red[w * GRP + tid];
+        Lh[tid] = L;
+        Wt[tid] = wt;
+    }
+    if (tid < G * NQ) {
+        const int q = tid % NQ, pg = tid / NQ;
+        const int h2 = q / (D / 4), d4 = q % (D / 4);
+        float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int p = pg; p < P; p += G) {
+            const float wgt = wts[p * GRP + h2];
+            if (wgt == 0.f) continue;
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.partials + (size_t)(wf + p + unit) * GRP * SR +
+                                                                     h2 * SR + 4) + d4);
+            s4.x = fmaf(v.x, wgt, s4.x);
+            s4.y = fmaf(v.y, wgt, s4.y);
+            s4.z = fmaf(v.z, wgt, s4.z);
+            s4.w = fmaf(v.w, wgt, s4.w);
+        }
+        acc4[pg * NQ + q] = s4;
+    }
+    __syncthreads();
+    if (tid < NQ) {
+        const int h2 = tid / (D / 4), d4 = tid % (D / 4);
+        float4 s4 = acc4[tid];
+        for (int pg = 1; pg < G; ++pg) {
+            const float4 v = acc4[pg * NQ + tid];
+            s4.x += v.x; s4.y += v.y; s4.z += v.z; s4.w += v.w;
+        }
+        const float L = Lh[h2];
+        const float linv = L > 0.f ? 1.f / L : 0.f;
+        *reinterpret_cast<float4 *>(obuf + h2 * D + 4 * d4) = make_float4(s4.x * linv, s4.y * linv, s4.z * linv,
+                                                                          s4.w * linv);
+        const float wt = Wt[h2];
+        float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (wt > 0.f) {
+            t4 = __ldcg(reinterpret_cast<const float4 *>(tl + h2 * SR + 4) + d4);
+            const float f = wt * linv;
+            t4.x *= f; t4.y *= f; t4.z *= f; t4.w *= f;
+        }
+        *reinterpret_cast<float4 *>(otl + h2 * D + 4 * d4) = t4;
+    }
+    __syncthreads();
+    if (warp < GRP) warp_fwht<D>(obuf + warp * D, 1, hb);
+    __syncthreads();
+    float *out = a.out + (size_t)unit * GRP * D;
+    for (int i = tid; i < GRP * D; i += NT) out[i] = obuf[i] + otl[i];
+    __syncthreads();  // the scratch is free again
 }
 
 template <int D, int GRP, typename Tin>
-static cudaError_t launch_dec(const DecodeArgs &a, int hb, cudaStream_t st)
+__global__ void __launch_bounds__(dec_warps<D, GRP>() * 32, 1)
+decode_kernel(DecodeArgs a, int hb)
+{
+    using R = Record<D>;
+    constexpr int W = dec_warps<D, GRP>();
+    constexpr int NNT = D / 8;
+    constexpr int C = 8 / GRP;
+    constexpr int SR = slot_row<D>();
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    DecWarpSmem<D, GRP> &sm = reinterpret_cast<DecWarpSmem<D, GRP> *>(smem_raw)[warp];
+    const int gl = lane >> 2, tig = lane & 3;
+    const int copy = gl / GRP, h = gl % GRP;
+
+    const long long nw = (long long)gridDim.x * W;
+    const long long per_unit = a.max_tokens / kBlockTokens + 1;  // blocks, then the tail item
+    const long long total = (long long)a.num_units * per_unit;
+    const long long wg = (long long)blockIdx.x * W + warp;
+    const long long i_begin = part_begin(wg, total, nw), i_end = part_begin(wg + 1, total, nw);
+
+    if (lane == 0) {
+        mbar_init(&sm.mbar[0]);
+        mbar_init(&sm.mbar[1]);
+    }
+    __syncwarp();
+    uint32_t kph = 0u, vph = 0u;
+    bool dead = false;  // a staged copy timed out: no more TMA from this warp
+
+    for (long long i = i_begin; i < i_end;) {
+        const int unit = (int)(i / per_unit);
+        const long long ibase = (long long)unit * per_unit;
+        const long long seg_end = min(i_end, ibase + per_unit);
+        const int s = unit / a.num_kv_heads;
+        int n = a.n_tokens[s];
+        if (n > a.max_tokens) {
+            if (lane == 0 && i == ibase) status_or(a.status, KVARN_STATUS_LENGTH);
+            n = a.max_tokens;
+        }
+        if (n < 0) n = 0;
+        const int nblk = n / kBlockTokens;
+        const int ntail = n - nblk * kBlockTokens;
+        const int b0 = (int)(i - ibase);
+        const int b1 = min((int)(seg_end - ibase), (int)(per_unit - 1));
+        const int b1r = min(b1, nblk);  // blocks beyond the sequence's length are skipped
+        const bool has_tail = seg_end == ibase + per_unit;
+
+        float m_run = -INFINITY, l_run = 0.f;
+        float2 orun[NNT];
+#pragma unroll
+        for (int j = 0; j < NNT; ++j) orun[j] = f2(0.f, 0.f);
+        if (b0 < b1r && !dead) {
+            // rotated query of this GQA group, scaled by softmax scale * log2(e)
+            const Tin *qg = static_cast<const Tin *>(a.q) + (size_t)unit * GRP * D;
+            for (int j = lane; j < GRP * D; j += 32) (&sm.qbuf[0][0])[j] = In<Tin>::load1(qg + j) * a.scale_log2;
+            __syncwarp();
+            warp_fwht<D>(&sm.qbuf[0][0], GRP, hb);
+            const unsigned char *kbase =
+                static_cast<const unsigned char *>(a.k_records) + (size_t)unit * a.max_blocks * R::kBytes;
+            const unsigned char *vbase =
+                static_cast<const unsigned char *>(a.v_records) + (size_t)unit * a.max_blocks * R::kBytes;
+            if (!run_blocks<D, GRP, Tin>(sm, kbase, vbase, b0, b1r, kph, vph, m_run, l_run, orun)) {
+                dead = true;
+                if (lane == 0) status_or(a.status, KVARN_STATUS_TIMEOUT);
+                m_run = -INFINITY;
+                l_run = 0.f;
+#pragma unroll
+                for (int j = 0; j < NNT; ++j) orun[j] = f2(0.f, 0.f);
+            }
+        }
+        // ---- this segment's block partial: (m, l, o_rot) per head
+        {
+            float *pp = a.partials + ((size_t)(wg + unit) * GRP + h) * SR;
+            float lsum = l_run;
+            lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+            lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+            if (copy == 0 && tig == 0) { pp[0] = m_run; pp[1] = lsum; }
+#pragma unroll
+            for (int nt = 0; nt < NNT; ++nt) {
+                if ((nt / (kGroup / 8)) % C == copy)
+                    *reinterpret_cast<float2 *>(pp + 4 + 8 * nt + 2 * tig) = orun[nt];
+            }
+        }
+        if (has_tail) tail_partial<D, GRP, Tin>(a, sm, unit, ntail, a.tail_partials + (size_t)unit * GRP * SR);
+
+        // ---- arrival: this segment's items are done
+        __syncwarp();
+        __threadfence();
+        uint32_t prev = 0u;
+        const uint32_t cnt = (uint32_t)(seg_end - i);
+        if (lane == 0) prev = atomicAdd(a.tickets + unit, cnt);
+        prev = __shfl_sync(0xffffffffu, prev, 0);
+        if (prev + cnt == (uint32_t)per_unit) {
+            __threadfence();
+            const long long wf = part_owner(ibase, total, nw), wl = part_owner(ibase + per_unit - 1, total, nw);
+            if (wl - wf + 1 <= kWarpMergeMax) {
+                warp_merge<D, GRP>(a, hb, sm, unit, wf, wl, total, nw);
+                if (lane == 0) a.tickets[unit] = 0u;
+            } else if (lane == 0) {
+                atomicExch(a.tickets + unit, kMergeFlag | blockIdx.x);
+            }
+        }
+        i = seg_end;
+    }
+
+    // ---- merges left to this CTA: units it touched whose ticket carries its
+    // mark.  Only a unit covered by more than kWarpMergeMax warps can carry
+    // one, and the CTA's contiguous range touches at most three of those (the
+    // first, one covered whole by at least kWarpMergeMax + 1 of its W warps,
+    // the last), so thread 0 lists them and every thread walks the same list.
+    __shared__ int merge_list[4];
+    __shared__ int merge_count;
+    __syncthreads();
+    const long long c_begin = part_begin((long long)blockIdx.x * W, total, nw);
+    const long long c_end = part_begin((long long)(blockIdx.x + 1) * W, total, nw);
+    if (threadIdx.x == 0) {
+        __threadfence();
+        int cnt = 0;
+        if (c_begin < c_end) {
+            const long long u_first = c_begin / per_unit, u_last = (c_end - 1) / per_unit;
+            for (long long unit = u_first; unit <= u_last && cnt < 4; ++unit) {
+                const long long ibase = unit * per_unit;
+                const long long span = part_owner(ibase + per_unit - 1, total, nw) - part_owner(ibase, total, nw) + 1;
+                if (span > kWarpMergeMax && __ldcg(a.tickets + unit) == (kMergeFlag | blockIdx.x))
+                    merge_list[cnt++] = (int)unit;
+            }
+        }
+        merge_count = cnt;
+    }
+    __syncthreads();
+    const int nmerge = merge_count;
+    for (int j = 0; j < nmerge; ++j) {
+        const int unit = merge_list[j];
+        const long long ibase = (long long)unit * per_unit;
+        const long long wf = part_owner(ibase, total, nw), wl = part_owner(ibase + per_unit - 1, total, nw);
+        cta_merge<D, GRP>(a, hb, smem_raw, unit, wf, wl, total, nw);
+        if (threadIdx.x == 0) a.tickets[unit] = 0u;
+    }
+}
+
+template <int D, int GRP, typename Tin>
+static cudaError_t launch_dec(const DecodeArgs &a, int hb, int ctas, cudaStream_t st)
 {
     constexpr int W = dec_warps<D, GRP>();
     const size_t smem = sizeof(DecWarpSmem<D, GRP>) * W;
+    // the CTA merge's scratch (see cta_merge) for the largest unit, covered by every warp
+    constexpr int NQ = GRP * D / 4, G = W * 32 / NQ;
+    const size_t merge = (size_t)G * NQ * 16 + 2 * (size_t)GRP * D * 4 + (size_t)((W * GRP + 3 * GRP + 3) & ~3) * 4 +
+                         (size_t)ctas * W * GRP * 4;
+    if (merge > smem) return cudaErrorInvalidConfiguration;
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, GRP, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    const int items = a.num_units * a.nsplit;
-    dim3 grid((unsigned)((items + W - 1) / W));
-    decode_kernel<D, GRP, Tin><<<grid, W * 32, smem, st>>>(a, hb);
+    decode_kernel<D, GRP, Tin><<<ctas, W * 32, smem, st>>>(a, hb);
     return cudaGetLastError();
 }
 
 template <int D, int GRP>
-static cudaError_t dispatch_dtype(int dtype, const DecodeArgs &a, int hb, cudaStream_t st)
+static cudaError_t dispatch_dtype(int dtype, const DecodeArgs &a, int hb, int ctas, cudaStream_t st)
 {
-    return dtype == KVARN_BF16 ? launch_dec<D, GRP, __nv_bfloat16>(a, hb, st) : launch_dec<D, GRP, float>(a, hb, st);
+    return dtype == KVARN_BF16 ? launch_dec<D, GRP, __nv_bfloat16>(a, hb, ctas, st)
+                               : launch_dec<D, GRP, float>(a, hb, ctas, st);
 }
 
 template <int D>
-static cudaError_t dispatch_grp(int dtype, const DecodeArgs &a, int hb, cudaStream_t st)
+static cudaError_t dispatch_grp(int dtype, const DecodeArgs &a, int hb, int ctas, cudaStream_t st)
 {
     switch (a.grp) {
-    case 1: return dispatch_dtype<D, 1>(dtype, a, hb, st);
-    case 2: return dispatch_dtype<D, 2>(dtype, a, hb, st);
-    case 4: return dispatch_dtype<D, 4>(dtype, a, hb, st);
-    case 8: return dispatch_dtype<D, 8>(dtype, a, hb, st);
+    case 1: return dispatch_dtype<D, 1>(dtype, a, hb, ctas, st);
+    case 2: return dispatch_dtype<D, 2>(dtype, a, hb, ctas, st);
+    case 4: return dispatch_dtype<D, 4>(dtype, a, hb, ctas, st);
+    case 8: return dispatch_dtype<D, 8>(dtype, a, hb, ctas, st);
     }
     return cudaErrorInvalidValue;
 }
 
-cudaError_t run_decode(const kvarn_config &c, const DecodeArgs &a, cudaStream_t st)
+cudaError_t run_decode(const kvarn_config &c, const DecodeArgs &a, int ctas, cudaStream_t st)
 {
     switch (c.head_dim) {
-    case 64: return dispatch_grp<64>(c.dtype, a, c.hadamard, st);
-    case 96: return dispatch_grp<96>(c.dtype, a, c.hadamard, st);
-    case 128: return dispatch_grp<128>(c.dtype, a, c.hadamard, st);
+    case 64: return dispatch_grp<64>(c.dtype, a, c.hadamard, ctas, st);
+    case 96: return dispatch_grp<96>(c.dtype, a, c.hadamard, ctas, st);
+    case 128: return dispatch_grp<128>(c.dtype, a, c.hadamard, ctas, st);
     }
     return cudaErrorInvalidValue;
 }
@@ -779,6 +1030,11 @@ static int warps_for(int grp)
 int decode_warps_per_cta(int head_dim, int grp)
 {
     return head_dim == 64 ? warps_for<64>(grp) : head_dim == 96 ? warps_for<96>(grp) : warps_for<128>(grp);
+}
+
+size_t decode_slot_bytes(int head_dim, int grp)
+{
+    return (size_t)grp * (head_dim + 4) * sizeof(float);
 }
 
 }  // namespace kvarn

@@ -98,7 +98,9 @@ size_t kvarn_decode_workspace_bytes(const kvarn_config *cfg, int num_q_heads)
         return 0;
     const int grp = num_q_heads / cfg->num_kv_heads;
     const size_t sh = (size_t)cfg->num_seqs * cfg->num_kv_heads;
-    return ticket_bytes(cfg) + sh * (kMaxSplits + 1) * grp * (cfg->head_dim + 2) * sizeof(float);
+    const size_t warps = (size_t)num_sms() * decode_warps_per_cta(cfg->head_dim, grp);
+    // tickets, one block partial per (warp, unit) segment (at most warps + units), one tail partial per unit
+    return ticket_bytes(cfg) + (warps + 2 * sh) * decode_slot_bytes(cfg->head_dim, grp);
 }
 
 int kvarn_quantize_blocks(const kvarn_config *cfg, const void *k, const void *v, int num_tokens,
@@ -159,17 +161,10 @@ int kvarn_decode_attention(const kvarn_config *cfg, const void *q, int num_q_hea
     const size_t need = kvarn_decode_workspace_bytes(cfg, num_q_heads);
     if (!workspace || !aligned16(workspace) || workspace_bytes < need) return KVARN_EWORKSPACE;
 
-    // one warp per (sequence, kv head, split); splits sized so that all warps
-    // are resident at once (one CTA of decode_warps_per_cta warps per SM)
+    // a persistent grid: one CTA of decode_warps_per_cta warps per SM, the
+    // item list (blocks and tails of all units) split evenly over the warps
     const int units = cfg->num_seqs * cfg->num_kv_heads;
-    const int nblk = max_tokens / cfg->block_tokens;
-    int nsplit = 1;
-    if (nblk > 0) {
-        int ns = num_sms() * decode_warps_per_cta(cfg->head_dim, grp) / units;
-        ns = ns < 1 ? 1 : ns;
-        ns = ns > nblk ? nblk : ns;
-        nsplit = ns > kMaxSplits ? kMaxSplits : ns;
-    }
+    const int ctas = num_sms();
     DecodeArgs a;
     a.q = q;
     a.k_records = cache->k_records; a.v_records = cache->v_records;
@@ -178,11 +173,13 @@ int kvarn_decode_attention(const kvarn_config *cfg, const void *q, int num_q_hea
     a.out = out;
     a.tickets = static_cast<uint32_t *>(workspace);
     a.partials = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + ticket_bytes(cfg));
+    a.tail_partials = a.partials + ((size_t)ctas * decode_warps_per_cta(cfg->head_dim, grp) + units) *
+                                       (decode_slot_bytes(cfg->head_dim, grp) / sizeof(float));
     const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)cfg->head_dim);
     a.scale_log2 = scale * 1.4426950408889634f;
     a.num_kv_heads = cfg->num_kv_heads; a.grp = grp; a.max_blocks = cfg->max_blocks;
-    a.max_tokens = max_tokens; a.num_units = units; a.nsplit = nsplit;
-    return cuda_status(run_decode(*cfg, a, static_cast<cudaStream_t>(stream)));
+    a.max_tokens = max_tokens; a.num_units = units;
+    return cuda_status(run_decode(*cfg, a, ctas, static_cast<cudaStream_t>(stream)));
 }
 
 int kvarn_dequantize(const kvarn_config *cfg, const kvarn_cache *cache, int first_block, int num_blocks,

@@ -73,6 +73,8 @@ struct In<float> {
         o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
         o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
     }
+    // load 4 consecutive elements (16 bytes, 16-byte aligned)
+    static __device__ __forceinline__ float4 load4(const float *p) { return __ldg(reinterpret_cast<const float4 *>(p)); }
     static __device__ __forceinline__ float load1(const float *p) { return *p; }
     static __device__ __forceinline__ void store1(float *p, float v) { *p = v; }
 };
@@ -88,6 +90,13 @@ struct In<__nv_bfloat16> {
             o[2 * i] = __uint_as_float(w[i] << 16);
             o[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
         }
+    }
+    // load 4 consecutive elements (8 bytes, 8-byte aligned) as fp32
+    static __device__ __forceinline__ float4 load4(const __nv_bfloat16 *p)
+    {
+        const uint2 a = __ldg(reinterpret_cast<const uint2 *>(p));
+        return make_float4(__uint_as_float(a.x << 16), __uint_as_float(a.x & 0xFFFF0000u),
+                           __uint_as_float(a.y << 16), __uint_as_float(a.y & 0xFFFF0000u));
     }
     static __device__ __forceinline__ float load1(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
     static __device__ __forceinline__ void store1(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }

@@ -42,24 +42,24 @@ struct DecodeArgs {
     const int32_t *n_tokens;
     int32_t *status;
     float *out;                 // [S][Hq][D]
-    float *partials;            // [S*Hkv][nsplit+1][grp][D+2]
-    uint32_t *tickets;          // [S*Hkv]
+    float *partials;            // [warps + units][grp][D+4]: one per (warp, unit) segment, at warp + unit
+    float *tail_partials;       // [units][grp][D+4]
+    uint32_t *tickets;          // [units], zero between calls
     float scale_log2;           // softmax scale * log2(e)
     int num_kv_heads, grp, max_blocks, max_tokens;
     int num_units;              // S * Hkv
-    int nsplit;                 // warps per unit; each takes a contiguous range of blocks
 };
 
 cudaError_t run_quantize(const kvarn_config &c, const QuantArgs &a, cudaStream_t st);
 cudaError_t run_append(const kvarn_config &c, const AppendArgs &a, cudaStream_t st);
 cudaError_t run_dequantize(const kvarn_config &c, const DequantArgs &a, cudaStream_t st);
-cudaError_t run_decode(const kvarn_config &c, const DecodeArgs &a, cudaStream_t st);
+cudaError_t run_decode(const kvarn_config &c, const DecodeArgs &a, int ctas, cudaStream_t st);
 cudaError_t run_set_length(int32_t *n_tokens, int num_seqs, int value, cudaStream_t st);
-
-// Largest split count the decode workspace is sized for.
-constexpr int kMaxSplits = 64;
 
 // Warps per decode CTA (one CTA per SM by shared memory).
 int decode_warps_per_cta(int head_dim, int grp);
+
+// Bytes of one decode partial (grp heads x (m, l, pad, pad, o[D])).
+size_t decode_slot_bytes(int head_dim, int grp);
 
 }  // namespace kvarn

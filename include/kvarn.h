@@ -142,10 +142,14 @@ KVARN_API size_t kvarn_cache_bytes(const kvarn_config *cfg, int part);
 
 /*
  * Workspace bytes kvarn_decode_attention needs for num_q_heads query heads
- * (split partial results and combine tickets).  Zero the workspace once
- * (e.g. cudaMemsetAsync) before its first use; every decode call leaves the
- * tickets zero again, so one workspace serves any number of calls that are
- * ordered on the GPU.
+ * on the current device: merge tickets (one uint32 per (sequence, kv head),
+ * padded to 256 bytes), then partial results -- one per (warp, sequence x kv
+ * head) segment of the persistent grid (at most SMs x warps per CTA + units)
+ * and one per unit for its residual tail, each grp x (D + 4) fp32.  The size
+ * depends on the device's SM count: query it on the device that runs the
+ * decode.  Zero the workspace once (e.g. cudaMemsetAsync) before its first
+ * use; every decode call leaves the tickets zero again, so one workspace
+ * serves any number of calls that are ordered on the GPU.
  */
 KVARN_API size_t kvarn_decode_workspace_bytes(const kvarn_config *cfg, int num_q_heads);
 
@@ -186,8 +190,10 @@ KVARN_API int kvarn_append_token(const kvarn_config *cfg, const void *k, const v
  * Query head h reads kv head h / (num_q_heads / num_kv_heads); num_q_heads
  * must be a multiple of num_kv_heads, at most 8 query heads per kv head.
  * softmax_scale <= 0 selects 1/sqrt(D).  max_tokens is an upper bound on
- * every n_tokens[s] (it sizes the split of the sequence across CTAs); a
- * sequence longer than that sets KVARN_STATUS_LENGTH and is cut to it.
+ * every n_tokens[s]: the work is split evenly over the warps of one CTA per
+ * SM as if every sequence held max_tokens tokens, so the closer the bound,
+ * the better the balance.  A sequence longer than that sets
+ * KVARN_STATUS_LENGTH and is cut to it.
  * A sequence with n_tokens 0 gets zeros.
  */
 KVARN_API int kvarn_decode_attention(const kvarn_config *cfg, const void *q, int num_q_heads,

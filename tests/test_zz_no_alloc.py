@@ -32,10 +32,11 @@ def test_noalloc_decode_matches_workspace_decode_twice_in_a_row():
 
 
 def test_noalloc_rejects_a_workspace_beyond_the_static_size():
-    cfg = kvarn.Config(8, 8, 128, max_blocks=1)  # 64 (sequence, kv head) pairs, GQA 8: ~17 MB of split partials
+    # 2048 (sequence, kv head) pairs at GQA 8: ~25 MB of partials (two 4 KB slots per pair, one per warp)
+    cfg = kvarn.Config(256, 8, 128, max_blocks=1)
     assert kvarn.decode_workspace_bytes(cfg, 64) > 16 << 20
     cache = kvarn.KVCache(cfg)
-    q = torch.zeros(8, 64, 128, dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros(256, 64, 128, dtype=torch.bfloat16, device="cuda")
     out = torch.zeros(q.shape, dtype=torch.float32, device="cuda")
     with pytest.raises(kvarn.KvarnError) as e:
         kvarn.decode_attention_noalloc(cfg, q, cache, 0, out)
