@@ -15,7 +15,7 @@
 //
 // B200 mapping.  The work of a launch is a list of items, unit by unit (a
 // unit is one (sequence, kv head)): the unit's max_tokens / 128 blocks, then
-// one item for its residual tail.  Every warp of a persistent grid (one CTA
+// kTailSlots items for its residual tail.  Every warp of a persistent grid (one CTA
 // per SM) takes an equal contiguous range of that list, so the load is even
 // whatever the number of units and their lengths relative to the SM count.
 // Where a range crosses into a new unit the warp starts a new online softmax.
@@ -59,7 +59,7 @@ constexpr long long kWaitLimit = 1LL << 26; // bounded mbarrier polling
 template <int D, int GRP>
 struct alignas(128) DecWarpSmem {
     unsigned char rec[2][Record<D>::kBytes];  // [K, V] of the current block
-    float scr[(D / kGroup) * kBlockTokens + kBlockTokens + D];
+    float scr[4 * kBlockTokens + kBlockTokens + D];  // K: srK[128][4], rK, cK; V: rsV[NG][128], rV, cV
     float qbuf[GRP][D];
     unsigned long long mbar[2];               // K record, V record
 };
@@ -247,27 +247,89 @@ __host__ __device__ constexpr int slot_row() { return D + 4; }
 
 // Partials are merged by the completing warp alone up to this many warps per unit.
 constexpr int kWarpMergeMax = 8;
+// Item slots of a unit's residual tail in the work list.  Attending up to 127
+// unrotated tokens on CUDA cores is a chain of dependent global loads, which
+// under the full streaming load costs about as much as three blocks; the
+// warp holding the first of these slots does it, the others have nothing to
+// do for them.
+constexpr int kTailSlots = 3;
 // Marker of a unit whose merge the completing warp left to its CTA.
 constexpr uint32_t kMergeFlag = 0x80000000u;
 
-// Blocks [b0, b1) of one unit into the running (m_run, l_run, orun).
-// Returns false if a staged copy did not arrive in time (after letting the
-// copies still in flight land, bounded); the warp then stops using TMA.
+// fp32 pair -> the fp16 pair of its high part (hl = 0) or of its remainder (hl = 1).
+__device__ __forceinline__ uint32_t hilo_part(float x, float y, bool hl)
+{
+    const __half2 hi = __floats2half2_rn(x, y);
+    const float2 hf = __half22float2(hi);
+    const __half2 lo = __floats2half2_rn(x - hf.x, y - hf.y);
+    return hl ? *reinterpret_cast<const uint32_t *>(&lo) : *reinterpret_cast<const uint32_t *>(&hi);
+}
+
+// K scales of one record to fp32, one lane per 4 consecutive tokens:
+// srK[t][g] = s[t][g] r[t] 2^16 (rows of 4, zero-padded), rK[t] = r[t], cK[d] = c[d].
+template <int D>
+__device__ __forceinline__ void convert_k_scales(const unsigned char *rec, float *srK, float *rK, float *cK)
+{
+    using R = Record<D>;
+    constexpr int NG = D / kGroup;
+    static_assert(NG <= 4, "score epilogue reads four groups per token");
+    const int lane = threadIdx.x & 31, t0 = 4 * lane;
+    const float4 r4 = h4_to_f4(reinterpret_cast<const uint2 *>(rec + R::kROff)[lane], 1.f);
+    *reinterpret_cast<float4 *>(rK + t0) = r4;
+    const uint2 *sp = reinterpret_cast<const uint2 *>(rec + R::kSOff) + lane * NG;
+    float sv[4 * NG];
+#pragma unroll
+    for (int i = 0; i < NG; ++i) {
+        const float4 f = h4_to_f4(sp[i], kTwo16);
+        sv[4 * i] = f.x; sv[4 * i + 1] = f.y; sv[4 * i + 2] = f.z; sv[4 * i + 3] = f.w;
+    }
+    const float rr[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float4 o;
+        o.x = sv[j * NG] * rr[j];
+        o.y = NG > 1 ? sv[j * NG + 1] * rr[j] : 0.f;
+        o.z = NG > 2 ? sv[j * NG + 2] * rr[j] : 0.f;
+        o.w = NG > 3 ? sv[j * NG + 3] * rr[j] : 0.f;
+        *reinterpret_cast<float4 *>(srK + 4 * (t0 + j)) = o;
+    }
+    const __half *ch = reinterpret_cast<const __half *>(rec + R::kCOff);
+    for (int d = lane; d < D; d += 32) cK[d] = __half2float(ch[d]);
+}
+
+// Blocks [b0, b1) of one unit into the running state.  Returns false if a
+// staged copy did not arrive in time (after letting the copies still in
+// flight land, bounded); the warp then stops using TMA.
+//
+// Scores (tensor cores): A = K codes of 16 tokens x 16 channels, B = q' of
+// 16 channels x 8 columns, a column per (head, hi/lo part) of four heads
+// (two n-tiles for eight); the accumulators of each 32-channel group take
+// their scale s r 2^16 in the epilogue, the m term is one more MMA with
+// A = m (tokens x groups) and B = Q (groups x columns).  A lane then holds
+// the scores of tokens 16u + gl and 16u + gl + 8 for head 4j + tig, so
+// m_run[j], l_run[j] (identical in the lanes of one tig) are those of that
+// head.  P V keeps the head-rows layout (A = p r s rows, B = V codes), whose
+// lanes get their probabilities from the score lanes by shuffles; orun is
+// in that layout (head gl % GRP).
 template <int D, int GRP, typename Tin>
 __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, const unsigned char *vbase, int b0,
-                           int b1, uint32_t &kph, uint32_t &vph, float &m_run, float &l_run, float2 (&orun)[D / 8])
+                           int b1, uint32_t &kph, uint32_t &vph, float (&m_run)[(GRP + 3) / 4],
+                           float (&l_run)[(GRP + 3) / 4], float2 (&orun)[D / 8])
 {
     using R = Record<D>;
     constexpr int NG = D / kGroup;          // channel groups
     constexpr int NKT = D / 16;             // k-tiles of the score MMA
     constexpr int NNT = D / 8;              // n-tiles of the P V MMA
-    constexpr int C = 8 / GRP;              // head copies in the 8 MMA rows
+    constexpr int C = 8 / GRP;              // head copies in the 8 rows of the P V MMA
     constexpr int SETS = (NG + C - 1) / C;  // groups handled per copy
     constexpr int KW = D / 32;              // K code words per (16-token unit, lane)
     constexpr int F = D / 64;
+    constexpr int NTN = (GRP + 3) / 4;      // score n-tiles (four heads each)
     const int lane = threadIdx.x & 31;
     const int gl = lane >> 2, tig = lane & 3;  // mma groupID, thread in group
-    const int copy = gl / GRP, h = gl % GRP;
+    const int copy = gl / GRP, h = gl % GRP;   // P V layout
+    const int hq = gl >> 1;                    // score B column: head 4j + hq, part hl
+    const bool hl = gl & 1;
 
     if (b0 >= b1) return true;
     if (lane == 0) {
@@ -286,137 +348,163 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
         const unsigned char *vrec = sm.rec[1];
         float *scr = sm.scr;
 
-        // ---- K scales to fp32: sK[g][t] = s * 2^16, rK[t], cK[d]
-        convert_scales<D, false>(krec, scr, scr + NG * kBlockTokens, scr + (NG + 1) * kBlockTokens, kTwo16, 1.f, 1.f);
+        // ---- K scales: srK[t][4] = s r 2^16, rK[t], cK[d]
+        float *srK = scr, *rK = scr + 4 * kBlockTokens, *cK = scr + 5 * kBlockTokens;
+        convert_k_scales<D>(krec, srK, rK, cK);
         __syncwarp();
-        const float *sK = scr, *rK = scr + NG * kBlockTokens, *cK = scr + (NG + 1) * kBlockTokens;
 
-        // ---- q' fragments (hi/lo rows) and the per-group sums Q_g
-        uint32_t Aq[NKT][4];
-        float Qg[NG];
+        // ---- q' B fragments (column part hl of head 4j + hq) and the group sums Q_g
+        uint32_t Bq[NTN][NKT][2];
+        uint32_t BQ[NTN];
 #pragma unroll
-        for (int g = 0; g < NG; ++g) Qg[g] = 0.f;
+        for (int j = 0; j < NTN; ++j) {
+            const int hh = 4 * j + hq;
+            const bool hv = hh < GRP;
+            const float *qh = sm.qbuf[hv ? hh : 0];
+            float Qg[NG];
 #pragma unroll
-        for (int kt = 0; kt < NKT; ++kt) {
-            const int k = 16 * kt + 2 * tig;
-            const float2 q01 = *reinterpret_cast<const float2 *>(&sm.qbuf[h][k]);
-            const float2 q89 = *reinterpret_cast<const float2 *>(&sm.qbuf[h][k + 8]);
-            const float v0 = q01.x * cK[k], v1 = q01.y * cK[k + 1];
-            const float v2 = q89.x * cK[k + 8], v3 = q89.y * cK[k + 9];
-            Qg[kt / 2] += (v0 + v1) + (v2 + v3);
-            const int g = kt / 2;
-            const bool mine = (g % C) == copy;
-            // channel block q = 2kt + cs sits at an even position for cs = 0
-            // (code scale 2^-16) and an odd one for cs = 1 (2^-18): times 4
-            if (mine) {
-                split_hilo(v0, v1, Aq[kt][0], Aq[kt][1]);
-                split_hilo(v2 * 4.f, v3 * 4.f, Aq[kt][2], Aq[kt][3]);
-            } else {
-                Aq[kt][0] = Aq[kt][1] = Aq[kt][2] = Aq[kt][3] = 0u;
+            for (int g = 0; g < NG; ++g) Qg[g] = 0.f;
+#pragma unroll
+            for (int kt = 0; kt < NKT; ++kt) {
+                const int k = 16 * kt + 2 * tig;
+                const float2 q01 = *reinterpret_cast<const float2 *>(qh + k);
+                const float2 q89 = *reinterpret_cast<const float2 *>(qh + k + 8);
+                const float2 c01 = *reinterpret_cast<const float2 *>(cK + k);
+                const float2 c89 = *reinterpret_cast<const float2 *>(cK + k + 8);
+                const float2 v01 = __fmul2_rn(q01, c01), v89 = __fmul2_rn(q89, c89);
+                Qg[kt / 2] += (v01.x + v01.y) + (v89.x + v89.y);
+                // channels 8..15 of a k-tile sit at odd code positions (scale 2^-18): times 4
+                Bq[j][kt][0] = hv ? hilo_part(v01.x, v01.y, hl) : 0u;
+                Bq[j][kt][1] = hv ? hilo_part(v89.x * 4.f, v89.y * 4.f, hl) : 0u;
             }
-        }
 #pragma unroll
-        for (int g = 0; g < NG; ++g) {
-            Qg[g] += __shfl_xor_sync(0xffffffffu, Qg[g], 1);
-            Qg[g] += __shfl_xor_sync(0xffffffffu, Qg[g], 2);
-        }
-        uint32_t AM[4] = {0u, 0u, 0u, 0u};  // M-term: rows = heads (copy 0), k = group
-        {
+            for (int g = 0; g < NG; ++g) {
+                Qg[g] += __shfl_xor_sync(0xffffffffu, Qg[g], 1);
+                Qg[g] += __shfl_xor_sync(0xffffffffu, Qg[g], 2);
+            }
             float q0 = 0.f, q1 = 0.f;
 #pragma unroll
             for (int g = 0; g < NG; ++g) {
                 if (g == 2 * tig) q0 = Qg[g];
                 if (g == 2 * tig + 1) q1 = Qg[g];
             }
-            if (copy == 0) split_hilo(q0, q1, AM[0], AM[1]);
+            BQ[j] = hv ? hilo_part(q0, q1, hl) : 0u;
         }
 
-        // ---- scores, 8 tokens per n-tile
-        float2 sc[16];
+        // ---- scores of tokens 16u + gl, 16u + gl + 8 for heads 4j + tig
+        float sc[NTN][8][2];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             CodeWord kw[KW];
             const uint32_t *wp = reinterpret_cast<const uint32_t *>(krec) + (u * 32 + lane) * KW;
 #pragma unroll
             for (int w = 0; w < KW; ++w) kw[w] = CodeWord(wp[w]);
-            // both 8-token n-tiles of the unit at once: independent MMA chains interleave
-            float acc[2][SETS][4];
+            float acc[NTN][NG][4];
 #pragma unroll
-            for (int ntl = 0; ntl < 2; ++ntl)
+            for (int j = 0; j < NTN; ++j)
 #pragma unroll
-                for (int st = 0; st < SETS; ++st) acc[ntl][st][0] = acc[ntl][st][1] = acc[ntl][st][2] = acc[ntl][st][3] = 0.f;
+                for (int g = 0; g < NG; ++g) acc[j][g][0] = acc[j][g][1] = acc[j][g][2] = acc[j][g][3] = 0.f;
 #pragma unroll
             for (int kt = 0; kt < NKT; ++kt) {
+                uint32_t aa[4];
 #pragma unroll
-                for (int ntl = 0; ntl < 2; ++ntl) {
-                    uint32_t bb[2];
+                for (int cs = 0; cs < 2; ++cs)
 #pragma unroll
-                    for (int cs = 0; cs < 2; ++cs) {
+                    for (int ntl = 0; ntl < 2; ++ntl) {
                         const int q = 2 * kt + cs;
                         int word, pos;
                         if (q < 8 * F) { word = ntl * F + q / 8; pos = q % 8; }
                         else { word = 2 * F; pos = q - 8 * F + 4 * ntl; }
-                        bb[cs] = code_pair(kw[word], pos);
+                        aa[2 * cs + ntl] = code_pair(kw[word], pos);
                     }
-                    mma16816(acc[ntl][(kt / 2) / C], Aq[kt], bb[0], bb[1]);
-                }
-            }
-            float accM[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-            for (int ntl = 0; ntl < 2; ++ntl) {
-                const int t = 16 * u + 8 * ntl + gl;
-                const __half *mh = reinterpret_cast<const __half *>(krec + R::kMOff) + t * NG;
-                uint32_t mp = 0u;
+                for (int j = 0; j < NTN; ++j) mma16816(acc[j][kt / 2], aa, Bq[j][kt][0], Bq[j][kt][1]);
+            }
+            // m term: A = m of tokens gl, gl + 8 and groups 2tig, 2tig + 1
+            uint32_t am[4] = {0u, 0u, 0u, 0u};
+            {
+                const __half *mh = reinterpret_cast<const __half *>(krec + R::kMOff);
+                const int ta = 16 * u + gl, tb = ta + 8;
                 if constexpr (NG % 2 == 0) {
-                    if (2 * tig < NG) mp = *reinterpret_cast<const uint32_t *>(mh + 2 * tig);
-                } else {
-                    const __half m0 = (2 * tig < NG) ? mh[2 * tig] : __float2half(0.f);
-                    const __half m1 = (2 * tig + 1 < NG) ? mh[2 * tig + 1] : __float2half(0.f);
-                    __half2 m2 = __halves2half2(m0, m1);
-                    mp = *reinterpret_cast<uint32_t *>(&m2);
-                }
-                mma16816(accM[ntl], AM, mp, 0u);
-            }
-#pragma unroll
-            for (int ntl = 0; ntl < 2; ++ntl) {
-                const int nt8 = 2 * u + ntl;
-                const int t0 = 8 * nt8 + 2 * tig;
-                float2 sum = hilo_sum(accM[ntl]);
-#pragma unroll
-                for (int st = 0; st < SETS; ++st) {
-                    const int g = st * C + copy;
-                    if (g < NG) {
-                        const float2 P = hilo_sum(acc[ntl][st]);
-                        const float2 sp = *reinterpret_cast<const float2 *>(sK + g * kBlockTokens + t0);
-                        sum = __ffma2_rn(P, sp, sum);
+                    if (2 * tig < NG) {
+                        am[0] = *reinterpret_cast<const uint32_t *>(mh + ta * NG + 2 * tig);
+                        am[1] = *reinterpret_cast<const uint32_t *>(mh + tb * NG + 2 * tig);
                     }
+                } else {
+                    const __half z = __float2half(0.f);
+                    __half2 pa = __halves2half2(2 * tig < NG ? mh[ta * NG + 2 * tig] : z,
+                                                2 * tig + 1 < NG ? mh[ta * NG + 2 * tig + 1] : z);
+                    __half2 pb = __halves2half2(2 * tig < NG ? mh[tb * NG + 2 * tig] : z,
+                                                2 * tig + 1 < NG ? mh[tb * NG + 2 * tig + 1] : z);
+                    am[0] = *reinterpret_cast<uint32_t *>(&pa);
+                    am[1] = *reinterpret_cast<uint32_t *>(&pb);
                 }
+            }
+            const float4 sra = *reinterpret_cast<const float4 *>(srK + 4 * (16 * u + gl));
+            const float4 srb = *reinterpret_cast<const float4 *>(srK + 4 * (16 * u + gl + 8));
+            const float ra = rK[16 * u + gl], rb = rK[16 * u + gl + 8];
+            const float swa[4] = {sra.x, sra.y, sra.z, sra.w}, swb[4] = {srb.x, srb.y, srb.z, srb.w};
 #pragma unroll
-                for (int cb = 1; cb < C; cb <<= 1) {
-                    sum.x += __shfl_xor_sync(0xffffffffu, sum.x, 4 * GRP * cb);
-                    sum.y += __shfl_xor_sync(0xffffffffu, sum.y, 4 * GRP * cb);
+            for (int j = 0; j < NTN; ++j) {
+                float accM[4] = {0.f, 0.f, 0.f, 0.f};
+                mma16816(accM, am, BQ[j], 0u);
+                float s0 = (accM[0] + accM[1]) * ra, s1 = (accM[2] + accM[3]) * rb;
+#pragma unroll
+                for (int g = 0; g < NG; ++g) {
+                    s0 = fmaf(acc[j][g][0] + acc[j][g][1], swa[g], s0);
+                    s1 = fmaf(acc[j][g][2] + acc[j][g][3], swb[g], s1);
                 }
-                sc[nt8] = __fmul2_rn(sum, *reinterpret_cast<const float2 *>(rK + t0));
+                sc[j][u][0] = s0;
+                sc[j][u][1] = s1;
             }
         }
 
-        // ---- online softmax (base 2; the scale carries log2(e))
-        float mb = -INFINITY;
+        // ---- online softmax (base 2; the scale carries log2(e)), per head 4j + tig
+        float alpha[NTN];
 #pragma unroll
-        for (int i2 = 0; i2 < 16; ++i2) mb = fmaxf(mb, fmaxf(sc[i2].x, sc[i2].y));
-        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
-        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
-        const float mnew = fmaxf(m_run, mb);
-        const float alpha = exp2f(m_run - mnew);
-        float ls = 0.f;
+        for (int j = 0; j < NTN; ++j) {
+            float mb = -INFINITY;
 #pragma unroll
-        for (int i2 = 0; i2 < 16; ++i2) {
-            sc[i2].x = exp2f(sc[i2].x - mnew);
-            sc[i2].y = exp2f(sc[i2].y - mnew);
-            ls += sc[i2].x + sc[i2].y;
+            for (int u = 0; u < 8; ++u) mb = fmaxf(mb, fmaxf(sc[j][u][0], sc[j][u][1]));
+            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 4));
+            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 8));
+            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 16));
+            const float mnew = fmaxf(m_run[j], mb);
+            alpha[j] = exp2f(m_run[j] - mnew);
+            float ls = 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                sc[j][u][0] = exp2f(sc[j][u][0] - mnew);
+                sc[j][u][1] = exp2f(sc[j][u][1] - mnew);
+                ls += sc[j][u][0] + sc[j][u][1];
+            }
+            ls += __shfl_xor_sync(0xffffffffu, ls, 4);
+            ls += __shfl_xor_sync(0xffffffffu, ls, 8);
+            ls += __shfl_xor_sync(0xffffffffu, ls, 16);
+            l_run[j] = fmaf(l_run[j], alpha[j], ls);
+            m_run[j] = mnew;
         }
-        l_run = fmaf(l_run, alpha, ls);
-        m_run = mnew;
+        // ---- probabilities into the P V layout: head h, tokens 16ks + 2tig + {0, 1, 8, 9}
+        float pv[8][4];
+        const int src0 = 8 * tig + (h & 3), src1 = src0 + 4;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+            for (int j = 0; j < NTN; ++j) {
+                const float x0 = __shfl_sync(0xffffffffu, sc[j][ks][0], src0);
+                const float x1 = __shfl_sync(0xffffffffu, sc[j][ks][0], src1);
+                const float x8 = __shfl_sync(0xffffffffu, sc[j][ks][1], src0);
+                const float x9 = __shfl_sync(0xffffffffu, sc[j][ks][1], src1);
+                if (j == 0 || (h >> 2) == j) {
+                    pv[ks][0] = x0; pv[ks][1] = x1; pv[ks][2] = x8; pv[ks][3] = x9;
+                }
+            }
+        }
+        float alphaV = __shfl_sync(0xffffffffu, alpha[0], h & 3);
+        if constexpr (NTN > 1) {
+            const float a1 = __shfl_sync(0xffffffffu, alpha[NTN - 1], h & 3);
+            if (h >= 4) alphaV = a1;
+        }
         __syncwarp();  // every lane is done with the K record and the K scales
         if (lane == 0 && b + 1 < b1)
             issue_record(&sm.mbar[0], sm.rec[0], kbase + (size_t)(b + 1) * R::kBytes, R::kBytes);
@@ -447,8 +535,8 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
                 const int T0 = 16 * ks + 2 * tig, T1 = T0 + 8;
                 uint32_t Ab[4] = {0u, 0u, 0u, 0u};
                 if (copy == 0) {
-                    split_hilo(sc[2 * ks].x * rV[T0], sc[2 * ks].y * rV[T0 + 1], Ab[0], Ab[1]);
-                    split_hilo(sc[2 * ks + 1].x * rV[T1], sc[2 * ks + 1].y * rV[T1 + 1], Ab[2], Ab[3]);
+                    split_hilo(pv[ks][0] * rV[T0], pv[ks][1] * rV[T0 + 1], Ab[0], Ab[1]);
+                    split_hilo(pv[ks][2] * rV[T1], pv[ks][3] * rV[T1 + 1], Ab[2], Ab[3]);
                 }
                 uint32_t bb0 = 0u, bb1 = 0u;
                 if (gl < NG) {
@@ -464,7 +552,7 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
 
         // ---- P V, one group set at a time
 #pragma unroll
-        for (int i2 = 0; i2 < NNT; ++i2) orun[i2] = __fmul2_rn(orun[i2], f2(alpha, alpha));
+        for (int i2 = 0; i2 < NNT; ++i2) orun[i2] = __fmul2_rn(orun[i2], f2(alphaV, alphaV));
 #pragma unroll
         for (int st = 0; st < SETS; ++st) {
             const int g = st * C + copy;
@@ -476,7 +564,8 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
                 if (gv) {
                     const float2 r0 = *reinterpret_cast<const float2 *>(rsV + g * kBlockTokens + T0);
                     const float2 r1 = *reinterpret_cast<const float2 *>(rsV + g * kBlockTokens + T1);
-                    const float2 p0 = __fmul2_rn(sc[2 * ks], r0), p1 = __fmul2_rn(sc[2 * ks + 1], r1);
+                    const float2 p0 = __fmul2_rn(f2(pv[ks][0], pv[ks][1]), r0);
+                    const float2 p1 = __fmul2_rn(f2(pv[ks][2], pv[ks][3]), r1);
                     split_hilo(p0.x, p0.y, Av[ks][0], Av[ks][1]);
                     split_hilo(p1.x, p1.y, Av[ks][2], Av[ks][3]);
                 } else {
@@ -541,59 +630,48 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
 }
 
 // The residual tail of one unit: unrotated query, CUDA cores.  Writes the
-// tail partial (m, l, o per head, unrotated basis) to dst.
+// tail partial (m, l, o per head, unrotated basis) to dst.  The tail is at
+// most 127 tokens and its cost is latency: every loop keeps a whole row (K)
+// or 16 rows (V) of loads in flight.
 template <int D, int GRP, typename Tin>
 __device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int unit, int ntail, float *dst)
 {
-    constexpr int QC = D / 4;   // channels per quarter of a row
-    constexpr int QP = QC + 4;  // padded quarter stride: the four quarters sit in different banks
     constexpr int SR = slot_row<D>();
+    constexpr int VB = 16;  // V rows per batch of loads
     const int lane = threadIdx.x & 31;
     float *ps = reinterpret_cast<float *>(sm.rec[0]);  // [128][GRP] scores, then weights
-    float *qt = ps + kBlockTokens * GRP;               // [GRP][4][QP] query, scaled
-    static_assert(sizeof(float) * (kBlockTokens * GRP + GRP * 4 * QP) <= sizeof(sm.rec), "tail scratch");
+    float *qt = ps + kBlockTokens * GRP;               // [GRP][D] query, scaled (uniform reads: broadcasts)
+    static_assert(sizeof(float) * (kBlockTokens * GRP + GRP * D) <= sizeof(sm.rec), "tail scratch");
     const Tin *qg = static_cast<const Tin *>(a.q) + (size_t)unit * GRP * D;
-    for (int i = lane; i < GRP * D; i += 32) {
-        const int hh = i / D, d = i % D;
-        qt[(hh * 4 + d / QC) * QP + d % QC] = In<Tin>::load1(qg + i) * a.scale_log2;
-    }
+    for (int i = lane; i < GRP * D; i += 32) qt[i] = In<Tin>::load1(qg + i) * a.scale_log2;
     __syncwarp();
-    // scores: 8 tokens at a time, lane = (token, quarter); the quarters are summed by shuffles
+    // scores: lanes over tokens, a row's loads issued together
     const Tin *kt = static_cast<const Tin *>(a.k_tail) + (size_t)unit * kBlockTokens * D;
-    const int tt = lane >> 2, qq = lane & 3;
-    for (int t0 = 0; t0 < ntail; t0 += 8) {
-        const int t = t0 + tt;
-        float acc[GRP];
-#pragma unroll
-        for (int hh = 0; hh < GRP; ++hh) acc[hh] = 0.f;
+    for (int t0 = 0; t0 < ntail; t0 += 32) {
+        const int t = t0 + lane;
         if (t < ntail) {
-            float kv[QC];
+            float acc[GRP];
 #pragma unroll
-            for (int c8 = 0; c8 < QC; c8 += 8) {
+            for (int hh = 0; hh < GRP; ++hh) acc[hh] = 0.f;
+            float kv[D];
+#pragma unroll
+            for (int c8 = 0; c8 < D; c8 += 8) {
                 float k8[8];
-                In<Tin>::load8(kt + (size_t)t * D + qq * QC + c8, k8);
+                In<Tin>::load8(kt + (size_t)t * D + c8, k8);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) kv[c8 + e] = k8[e];
             }
 #pragma unroll
-            for (int hh = 0; hh < GRP; ++hh) {
-                const float *qr = qt + (hh * 4 + qq) * QP;
+            for (int c4 = 0; c4 < D; c4 += 4) {
 #pragma unroll
-                for (int c4 = 0; c4 < QC; c4 += 4) {
-                    const float4 qv = *reinterpret_cast<const float4 *>(qr + c4);
+                for (int hh = 0; hh < GRP; ++hh) {
+                    const float4 qv = *reinterpret_cast<const float4 *>(qt + hh * D + c4);
                     acc[hh] = fmaf(qv.x, kv[c4], acc[hh]);
                     acc[hh] = fmaf(qv.y, kv[c4 + 1], acc[hh]);
                     acc[hh] = fmaf(qv.z, kv[c4 + 2], acc[hh]);
                     acc[hh] = fmaf(qv.w, kv[c4 + 3], acc[hh]);
                 }
             }
-        }
-#pragma unroll
-        for (int hh = 0; hh < GRP; ++hh) {
-            acc[hh] += __shfl_xor_sync(0xffffffffu, acc[hh], 1);
-            acc[hh] += __shfl_xor_sync(0xffffffffu, acc[hh], 2);
-        }
-        if (qq == 0 && t < ntail) {
 #pragma unroll
             for (int hh = 0; hh < GRP; ++hh) ps[t * GRP + hh] = acc[hh];
         }
@@ -626,29 +704,30 @@ __device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int u
         lt[hh] = sum;
     }
     __syncwarp();
-    // P V: lanes over channel quads, eight tokens' loads in flight
+    // P V: lanes over channel quads, VB rows' loads in flight
     const Tin *vt = static_cast<const Tin *>(a.v_tail) + (size_t)unit * kBlockTokens * D;
     const int c0 = 4 * lane;
     const bool act = c0 < D;
     float4 o[GRP];
 #pragma unroll
     for (int hh = 0; hh < GRP; ++hh) o[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int t0 = 0; t0 < ntail; t0 += 8) {
-        float4 vv[8];
+    for (int t0 = 0; t0 < ntail; t0 += VB) {
+        typename In<Tin>::Raw4 vr[VB];
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-            vv[u] = (act && t0 + u < ntail) ? In<Tin>::load4(vt + (size_t)(t0 + u) * D + c0)
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < VB; ++u)
+            vr[u] = In<Tin>::load4_raw(vt + (size_t)min(t0 + u, ntail - 1) * D + (act ? c0 : 0));
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            if (t0 + u >= ntail) break;
+        for (int u = 0; u < VB; ++u) {
+            if (act && t0 + u < ntail) {
+                const float4 vv = In<Tin>::widen4(vr[u]);
 #pragma unroll
-            for (int hh = 0; hh < GRP; ++hh) {
-                const float p = ps[(t0 + u) * GRP + hh];
-                o[hh].x = fmaf(p, vv[u].x, o[hh].x);
-                o[hh].y = fmaf(p, vv[u].y, o[hh].y);
-                o[hh].z = fmaf(p, vv[u].z, o[hh].z);
-                o[hh].w = fmaf(p, vv[u].w, o[hh].w);
+                for (int hh = 0; hh < GRP; ++hh) {
+                    const float p = ps[(t0 + u) * GRP + hh];
+                    o[hh].x = fmaf(p, vv.x, o[hh].x);
+                    o[hh].y = fmaf(p, vv.y, o[hh].y);
+                    o[hh].z = fmaf(p, vv.z, o[hh].z);
+                    o[hh].w = fmaf(p, vv.w, o[hh].w);
+                }
             }
         }
     }
@@ -719,7 +798,8 @@ __device__ void warp_merge(const DecodeArgs &a, int hb, DecWarpSmem<D, GRP> &sm,
 
 // Merge of one unit by all warps of the CTA (many partials).  Every thread
 // of the CTA calls it with the same arguments; the whole dynamic shared
-// memory is scratch.
+// memory is scratch.  A slot of a warp whose range is empty was never
+// written: it is neither read nor weighted.
 template <int D, int GRP>
 __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int unit, long long wf, long long wl,
                           long long total, long long nw)
@@ -729,10 +809,12 @@ __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int 
     constexpr int SR = slot_row<D>();
     constexpr int NQ = GRP * D / 4;  // float4 columns of a unit's output
     constexpr int G = NT / NQ;       // partial groups summed in parallel
+    constexpr int UN = 8;            // partial loads in flight per thread
     static_assert(G >= 1, "merge layout");
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int P = (int)(wl - wf + 1);
     const float *tl = a.tail_partials + (size_t)unit * GRP * SR;
+    const float *slots = a.partials + (size_t)(wf + unit) * GRP * SR;  // slot of warp wf + p at p * GRP * SR
 
     // scratch, every array starting on a 16-byte boundary
     constexpr int SMALL = (W * GRP + 3 * GRP + 3) & ~3;      // red [W][GRP], Mh, Lh, Wt [GRP]
@@ -743,14 +825,19 @@ __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int 
     float *Mh = red + W * GRP;
     float *Lh = Mh + GRP;
     float *Wt = Lh + GRP;
-    float *wts = red + SMALL;                                // [P][GRP]
+    float2 *ml = reinterpret_cast<float2 *>(red + SMALL);    // [P][GRP] (m, l); m = -inf for an empty warp
+    float *wts = reinterpret_cast<float *>(ml + P * GRP);    // [P][GRP]
 
+    // (m, l) of every partial and head, and the maximum per head
     const int hh = tid % GRP;  // NT is a multiple of 32, so every thread keeps one head
     float mx = -INFINITY;
     for (int idx = tid; idx < P * GRP; idx += NT) {
         const long long w = wf + idx / GRP;
+        float2 v = f2(-INFINITY, 0.f);
         if (part_begin(w, total, nw) < part_begin(w + 1, total, nw))
-            mx = fmaxf(mx, __ldcg(a.partials + (size_t)(w + unit) * GRP * SR + hh * SR));
+            v = __ldcg(reinterpret_cast<const float2 *>(slots + (size_t)(idx / GRP) * GRP * SR + hh * SR));
+        ml[idx] = v;
+        mx = fmaxf(mx, v.x);
     }
     for (int o = GRP; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     if (lane < GRP) red[warp * GRP + lane] = mx;
@@ -761,21 +848,43 @@ __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int 
         Mh[tid] = M;
     }
     __syncthreads();
+    // weights exp2(m - M) and the normaliser
     const float M = Mh[hh];
     float ls = 0.f;
     for (int idx = tid; idx < P * GRP; idx += NT) {
-        const long long w = wf + idx / GRP;
-        float wgt = 0.f;
-        if (M > -INFINITY && part_begin(w, total, nw) < part_begin(w + 1, total, nw)) {
-            const float *row = a.partials + (size_t)(w + unit) * GRP * SR + hh * SR;
-            wgt = exp2f(__ldcg(row) - M);
-            ls = fmaf(__ldcg(row + 1), wgt, ls);
-        }
+        const float2 v = ml[idx];
+        const float wgt = (M > -INFINITY && v.x > -INFINITY) ? exp2f(v.x - M) : 0.f;
         wts[idx] = wgt;
+        ls = fmaf(v.y, wgt, ls);
     }
     for (int o = GRP; o < 32; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-    __syncthreads();  // every thread has read red
+    __syncthreads();  // every thread has read red and written wts
     if (lane < GRP) red[warp * GRP + lane] = ls;
+    // the weighted sum of the o rows: threads over (group of partials, float4 column)
+    if (tid < G * NQ) {
+        const int q = tid % NQ, pg = tid / NQ;
+        const int h2 = q / (D / 4), d4 = q % (D / 4);
+        float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int p0 = pg; p0 < P; p0 += G * UN) {
+            float4 v[UN];
+            float wv[UN];
+#pragma unroll
+            for (int u = 0; u < UN; ++u) {
+                const int p = p0 + u * G;
+                wv[u] = p < P ? wts[p * GRP + h2] : 0.f;
+                v[u] = wv[u] != 0.f ? __ldcg(reinterpret_cast<const float4 *>(slots + (size_t)p * GRP * SR + h2 * SR + 4) + d4)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < UN; ++u) {
+                s4.x = fmaf(v[u].x, wv[u], s4.x);
+                s4.y = fmaf(v[u].y, wv[u], s4.y);
+                s4.z = fmaf(v[u].z, wv[u], s4.z);
+                s4.w = fmaf(v[u].w, wv[u], s4.w);
+            }
+        }
+        acc4[pg * NQ + q] = s4;
+    }
     __syncthreads();
     if (tid < GRP) {
         const float Mt = Mh[tid];
@@ -784,22 +893,6 @@ __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int 
         for (int w = 0; w < W; ++w) L += red[w * GRP + tid];
         Lh[tid] = L;
         Wt[tid] = wt;
-    }
-    if (tid < G * NQ) {
-        const int q = tid % NQ, pg = tid / NQ;
-        const int h2 = q / (D / 4), d4 = q % (D / 4);
-        float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int p = pg; p < P; p += G) {
-            const float wgt = wts[p * GRP + h2];
-            if (wgt == 0.f) continue;
-            const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.partials + (size_t)(wf + p + unit) * GRP * SR +
-                                                                     h2 * SR + 4) + d4);
-            s4.x = fmaf(v.x, wgt, s4.x);
-            s4.y = fmaf(v.y, wgt, s4.y);
-            s4.z = fmaf(v.z, wgt, s4.z);
-            s4.w = fmaf(v.w, wgt, s4.w);
-        }
-        acc4[pg * NQ + q] = s4;
     }
     __syncthreads();
     if (tid < NQ) {
@@ -830,6 +923,18 @@ __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int 
     __syncthreads();  // the scratch is free again
 }
 
+// Most partials the CTA merge holds in shared memory: beyond that (only when
+// a unit is spread over nearly the whole grid at the largest GQA groups) the
+// completing warp merges alone.
+template <int D, int GRP>
+__host__ __device__ constexpr int cta_merge_max()
+{
+    constexpr int W = dec_warps<D, GRP>();
+    constexpr int NQ = GRP * D / 4, G = W * 32 / NQ;
+    constexpr int fixed = G * NQ * 16 + 2 * GRP * D * 4 + ((W * GRP + 3 * GRP + 3) & ~3) * 4;
+    return (int)((sizeof(DecWarpSmem<D, GRP>) * W - fixed) / (GRP * 12));
+}
+
 template <int D, int GRP, typename Tin>
 __global__ void __launch_bounds__(dec_warps<D, GRP>() * 32, 1)
 decode_kernel(DecodeArgs a, int hb)
@@ -838,6 +943,7 @@ decode_kernel(DecodeArgs a, int hb)
     constexpr int W = dec_warps<D, GRP>();
     constexpr int NNT = D / 8;
     constexpr int C = 8 / GRP;
+    constexpr int NTN = (GRP + 3) / 4;
     constexpr int SR = slot_row<D>();
     extern __shared__ __align__(128) unsigned char smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -846,7 +952,8 @@ decode_kernel(DecodeArgs a, int hb)
     const int copy = gl / GRP, h = gl % GRP;
 
     const long long nw = (long long)gridDim.x * W;
-    const long long per_unit = a.max_tokens / kBlockTokens + 1;  // blocks, then the tail item
+    const int nb_max = a.max_tokens / kBlockTokens;
+    const long long per_unit = nb_max + kTailSlots;  // blocks, then the tail's slots
     const long long total = (long long)a.num_units * per_unit;
     const long long wg = (long long)blockIdx.x * W + warp;
     const long long i_begin = part_begin(wg, total, nw), i_end = part_begin(wg + 1, total, nw);
@@ -873,11 +980,13 @@ decode_kernel(DecodeArgs a, int hb)
         const int nblk = n / kBlockTokens;
         const int ntail = n - nblk * kBlockTokens;
         const int b0 = (int)(i - ibase);
-        const int b1 = min((int)(seg_end - ibase), (int)(per_unit - 1));
+        const int b1 = (int)min(seg_end - ibase, (long long)nb_max);
         const int b1r = min(b1, nblk);  // blocks beyond the sequence's length are skipped
-        const bool has_tail = seg_end == ibase + per_unit;
+        const bool has_tail = i - ibase <= nb_max && seg_end - ibase > nb_max;
 
-        float m_run = -INFINITY, l_run = 0.f;
+        float m_run[NTN], l_run[NTN];
+#pragma unroll
+        for (int j = 0; j < NTN; ++j) { m_run[j] = -INFINITY; l_run[j] = 0.f; }
         float2 orun[NNT];
 #pragma unroll
         for (int j = 0; j < NNT; ++j) orun[j] = f2(0.f, 0.f);
@@ -894,19 +1003,23 @@ decode_kernel(DecodeArgs a, int hb)
             if (!run_blocks<D, GRP, Tin>(sm, kbase, vbase, b0, b1r, kph, vph, m_run, l_run, orun)) {
                 dead = true;
                 if (lane == 0) status_or(a.status, KVARN_STATUS_TIMEOUT);
-                m_run = -INFINITY;
-                l_run = 0.f;
+#pragma unroll
+                for (int j = 0; j < NTN; ++j) { m_run[j] = -INFINITY; l_run[j] = 0.f; }
 #pragma unroll
                 for (int j = 0; j < NNT; ++j) orun[j] = f2(0.f, 0.f);
             }
         }
         // ---- this segment's block partial: (m, l, o_rot) per head
         {
-            float *pp = a.partials + ((size_t)(wg + unit) * GRP + h) * SR;
-            float lsum = l_run;
-            lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
-            lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
-            if (copy == 0 && tig == 0) { pp[0] = m_run; pp[1] = lsum; }
+            float *slot = a.partials + (size_t)(wg + unit) * GRP * SR;
+            // (m, l) of head 4j + tig sit in every lane of that tig
+#pragma unroll
+            for (int j = 0; j < NTN; ++j)
+                if (gl == 0 && 4 * j + tig < GRP) {
+                    slot[(4 * j + tig) * SR] = m_run[j];
+                    slot[(4 * j + tig) * SR + 1] = l_run[j];
+                }
+            float *pp = slot + h * SR;
 #pragma unroll
             for (int nt = 0; nt < NNT; ++nt) {
                 if ((nt / (kGroup / 8)) % C == copy)
@@ -925,7 +1038,8 @@ decode_kernel(DecodeArgs a, int hb)
         if (prev + cnt == (uint32_t)per_unit) {
             __threadfence();
             const long long wf = part_owner(ibase, total, nw), wl = part_owner(ibase + per_unit - 1, total, nw);
-            if (wl - wf + 1 <= kWarpMergeMax) {
+            const long long span = wl - wf + 1;
+            if (span <= kWarpMergeMax || span > cta_merge_max<D, GRP>()) {
                 warp_merge<D, GRP>(a, hb, sm, unit, wf, wl, total, nw);
                 if (lane == 0) a.tickets[unit] = 0u;
             } else if (lane == 0) {
@@ -936,8 +1050,8 @@ decode_kernel(DecodeArgs a, int hb)
     }
 
     // ---- merges left to this CTA: units it touched whose ticket carries its
-    // mark.  Only a unit covered by more than kWarpMergeMax warps can carry
-    // one, and the CTA's contiguous range touches at most three of those (the
+    // mark.  Only a unit covered by more than kWarpMergeMax warps (and at most
+    // cta_merge_max) can carry one, and the CTA's contiguous range touches at most three of those (the
     // first, one covered whole by at least kWarpMergeMax + 1 of its W warps,
     // the last), so thread 0 lists them and every thread walks the same list.
     __shared__ int merge_list[4];
@@ -953,7 +1067,8 @@ decode_kernel(DecodeArgs a, int hb)
             for (long long unit = u_first; unit <= u_last && cnt < 4; ++unit) {
                 const long long ibase = unit * per_unit;
                 const long long span = part_owner(ibase + per_unit - 1, total, nw) - part_owner(ibase, total, nw) + 1;
-                if (span > kWarpMergeMax && __ldcg(a.tickets + unit) == (kMergeFlag | blockIdx.x))
+                if (span > kWarpMergeMax && span <= cta_merge_max<D, GRP>() &&
+                    __ldcg(a.tickets + unit) == (kMergeFlag | blockIdx.x))
                     merge_list[cnt++] = (int)unit;
             }
         }
@@ -975,11 +1090,6 @@ static cudaError_t launch_dec(const DecodeArgs &a, int hb, int ctas, cudaStream_
 {
     constexpr int W = dec_warps<D, GRP>();
     const size_t smem = sizeof(DecWarpSmem<D, GRP>) * W;
-    // the CTA merge's scratch (see cta_merge) for the largest unit, covered by every warp
-    constexpr int NQ = GRP * D / 4, G = W * 32 / NQ;
-    const size_t merge = (size_t)G * NQ * 16 + 2 * (size_t)GRP * D * 4 + (size_t)((W * GRP + 3 * GRP + 3) & ~3) * 4 +
-                         (size_t)ctas * W * GRP * 4;
-    if (merge > smem) return cudaErrorInvalidConfiguration;
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, GRP, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;

@@ -75,6 +75,10 @@ struct In<float> {
     }
     // load 4 consecutive elements (16 bytes, 16-byte aligned)
     static __device__ __forceinline__ float4 load4(const float *p) { return __ldg(reinterpret_cast<const float4 *>(p)); }
+    // the same as raw bits, widened later (fewer registers while loads are in flight)
+    using Raw4 = float4;
+    static __device__ __forceinline__ Raw4 load4_raw(const float *p) { return load4(p); }
+    static __device__ __forceinline__ float4 widen4(Raw4 r) { return r; }
     static __device__ __forceinline__ float load1(const float *p) { return *p; }
     static __device__ __forceinline__ void store1(float *p, float v) { *p = v; }
 };
@@ -95,6 +99,16 @@ struct In<__nv_bfloat16> {
     static __device__ __forceinline__ float4 load4(const __nv_bfloat16 *p)
     {
         const uint2 a = __ldg(reinterpret_cast<const uint2 *>(p));
+        return make_float4(__uint_as_float(a.x << 16), __uint_as_float(a.x & 0xFFFF0000u),
+                           __uint_as_float(a.y << 16), __uint_as_float(a.y & 0xFFFF0000u));
+    }
+    using Raw4 = uint2;
+    static __device__ __forceinline__ Raw4 load4_raw(const __nv_bfloat16 *p)
+    {
+        return __ldg(reinterpret_cast<const uint2 *>(p));
+    }
+    static __device__ __forceinline__ float4 widen4(Raw4 a)
+    {
         return make_float4(__uint_as_float(a.x << 16), __uint_as_float(a.x & 0xFFFF0000u),
                            __uint_as_float(a.y << 16), __uint_as_float(a.y & 0xFFFF0000u));
     }
