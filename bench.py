@@ -38,6 +38,10 @@ WORKLOAD = ("Qwen3-4B-shaped long-horizon decode: batch 8, 32 q / 8 kv heads, he
             "36 layer caches, context 32641..32768 (one 128-token block period per step: 128 x 36 x "
             "(append+quantise-on-fill, decode attention))")
 QB_WORKLOAD = "Llama-3-8B-shaped bulk prefill quantise: 32 batch x 32 layers x 8 kv heads x 8192 tokens x 128, bf16"
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one decode launch at context 32705 for this
+# batch, from one ncu capture of `bench.py --profile decode` with the current decode kernel; reset it to None
+# whenever the decode kernel changes until it is captured again.
+DECODE_TRAFFIC_BYTES = 219942400 + 4037888
 
 
 def _peaks():
@@ -439,7 +443,7 @@ def main():
                        "parallelism": f"dp{world} (independent batches, no collective)",
                        "l2": "inputs larger than L2: each decode launch streams ~219 MB of cache, 7.9 GB per token"},
             "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": r["achieved"], "peak": r["peak"],
-                         "unit": "GB/s", "frac": r["achieved"] / r["peak"], "traffic": None,
+                         "unit": "GB/s", "frac": r["achieved"] / r["peak"], "traffic": DECODE_TRAFFIC_BYTES,
                          "peak_source": r["peak_kind"], "algorithmic_bytes_per_launch": r["dbytes"],
                          "launch_ms": r["dec_avg_ms"]},
             "e2e": {"value": r["e2e_value"], "unit": UNIT, "h2d_bytes_per_step": r["h2d"],
