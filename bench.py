@@ -251,9 +251,10 @@ def run_kvarn(args, world, rank, local):
     quant = None
     if not args.skip_quant:
         quant = run_bulk_quant(args, dev, seed, peak)
+    ablation = None if args.skip_ablation or rank != 0 else run_ablation(dev)
 
     return dict(value=value, ms_step=ms_step, clocks=clk, dec_avg_ms=dec_avg_ms, dbytes=dbytes, achieved=achieved,
-                peak=peak, peak_kind=peak_kind, e2e_value=e2e_value, h2d=h2d, d2h=d2h, quant=quant,
+                peak=peak, peak_kind=peak_kind, e2e_value=e2e_value, h2d=h2d, d2h=d2h, quant=quant, ablation=ablation,
                 launches=args.steps * T_BLK * LAYERS * 2)
 
 
@@ -352,6 +353,40 @@ def oracle_sample(max_threads: int = 16):
                        f"per token for the 8-sequence batch")
 
 
+# ------------------------------------------------------------------- ablation of the two stages
+def run_ablation(dev):
+    """Magnitude / direction error of the stored K and V per token, for the full encoding and with the rotation,
+    the normalisation or both switched off (one Qwen3-4B-shaped layer: 8 sequences x 8 kv heads x 4096 tokens,
+    bf16), measured by kvarn_token_errors on the GPU; plus that kernel's time."""
+    from bit_kv_cache_token_b200 import kvarn, synth
+    k, v = synth.layer_kv(9, 0, S, HKV, 4096, D, n_outliers=4, device=dev)
+    out = {}
+    for name, hb, sw in (("kvarn", D, 4), ("no_rotation", 0, 4), ("no_normalisation", D, 0), ("plain_rtn", 0, 0)):
+        cfg = kvarn.Config(S, HKV, D, max_blocks=4096 // T_BLK, hadamard=hb, sweeps=sw, dtype=kvarn.KVARN_BF16)
+        c = kvarn.KVCache(cfg, device=dev)
+        kvarn.quantize_blocks(cfg, k, v, c)
+        ek, ev = kvarn.token_errors(cfg, k, v, c)
+        torch.cuda.synchronize()
+        row = {}
+        for tn, e in (("k", ek), ("v", ev)):
+            e = e.reshape(-1, 2)
+            row[f"{tn}_magnitude_mean"] = float(e[:, 0].mean())
+            row[f"{tn}_direction_mean"] = float(e[:, 1].mean())
+            row[f"{tn}_magnitude_p99"] = float(torch.quantile(e[:, 0], 0.99))
+            row[f"{tn}_direction_p99"] = float(torch.quantile(e[:, 1], 0.99))
+        out[name] = row
+        if name == "kvarn":
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(10):
+                kvarn.token_errors(cfg, k, v, c)
+            e1.record()
+            torch.cuda.synchronize()
+            out["token_errors_ms"] = e0.elapsed_time(e1) / 10
+    out["workload"] = "Qwen3-4B-shaped layer: 8 sequences x 8 kv heads x 4096 tokens x 128, bf16"
+    return out
+
+
 # ------------------------------------------------------------------- small profiling cases
 def run_profile_case(case: str):
     """Small cases for ncu captures: 3 launches of one kernel on inputs larger than L2.
@@ -397,6 +432,7 @@ def main():
     ap.add_argument("--skip-quant", action="store_true", help="skip the bulk quantise measurement")
     ap.add_argument("--small", action="store_true", help="reduced bulk quantise size (quick checks)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-ablation", action="store_true", help="skip the rotation / normalisation ablation")
     ap.add_argument("--profile", choices=["decode", "quantize", "append"], default=None,
                     help="run a small case of one kernel for ncu and exit")
     args = ap.parse_args()
@@ -454,6 +490,8 @@ def main():
         if q:
             line["quantize"] = {"workload": q["workload"], "gbs": q["gbs"], "ms": q["ms"], "frac": q["frac"],
                                 "algorithmic_bytes": q["bytes"], "peak": r["peak"], "status": q["status"]}
+        if r["ablation"]:
+            line["ablation"] = r["ablation"]
         if cpu:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)

@@ -182,6 +182,26 @@ int kvarn_decode_attention(const kvarn_config *cfg, const void *q, int num_q_hea
     return cuda_status(run_decode(*cfg, a, ctas, static_cast<cudaStream_t>(stream)));
 }
 
+int kvarn_token_errors(const kvarn_config *cfg, const void *k, const void *v, int num_tokens, int first_block,
+                       const kvarn_cache *cache, float *err_k, float *err_v, void *stream)
+{
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if ((rc = check_cache(cache, false))) return rc;
+    if (num_tokens < 0 || num_tokens % cfg->block_tokens || first_block < 0) return KVARN_EINVAL;
+    const int nb = num_tokens / cfg->block_tokens;
+    if ((long long)first_block + nb > cfg->max_blocks) return KVARN_EINVAL;
+    if (nb == 0) return KVARN_OK;
+    if (!k || !v || !err_k || !err_v || !aligned16(k) || !aligned16(v) || !aligned16(err_k) || !aligned16(err_v))
+        return KVARN_EINVAL;
+    ErrorArgs a;
+    a.k = k; a.v = v;
+    a.k_records = cache->k_records; a.v_records = cache->v_records;
+    a.err_k = err_k; a.err_v = err_v;
+    a.num_blocks = nb; a.first_block = first_block; a.max_blocks = cfg->max_blocks;
+    return cuda_status(run_token_errors(*cfg, a, static_cast<cudaStream_t>(stream)));
+}
+
 int kvarn_dequantize(const kvarn_config *cfg, const kvarn_cache *cache, int first_block, int num_blocks,
                      int rotated, float *k_out, float *v_out, void *stream)
 {

@@ -50,7 +50,15 @@ struct DecodeArgs {
     int num_units;              // S * Hkv
 };
 
+struct ErrorArgs {
+    const void *k, *v;          // [S][Hkv][num_blocks * T][D], the rows that were quantised
+    const void *k_records, *v_records;
+    float *err_k, *err_v;       // [S][Hkv][num_blocks * T][2]: magnitude, direction
+    int num_blocks, first_block, max_blocks;
+};
+
 cudaError_t run_quantize(const kvarn_config &c, const QuantArgs &a, cudaStream_t st);
+cudaError_t run_token_errors(const kvarn_config &c, const ErrorArgs &a, cudaStream_t st);
 cudaError_t run_append(const kvarn_config &c, const AppendArgs &a, cudaStream_t st);
 cudaError_t run_dequantize(const kvarn_config &c, const DequantArgs &a, cudaStream_t st);
 cudaError_t run_decode(const kvarn_config &c, const DecodeArgs &a, int ctas, cudaStream_t st);

@@ -94,19 +94,14 @@ __device__ __forceinline__ void load_block(const Tin *rows, float2 (&X)[4][16])
     }
 }
 
-// Quantise the block held in X (destroyed) into rec_out (global, 16-byte
-// aligned, Record<D>::kBytes); TENSOR 0 = K code order, 1 = V code order.  dbg: NULL or fp32 [T + D + 2*T*D/32] unrounded
-// r, c, s, m.  All D threads of the CTA must call this.
-template <int D, int HB, int TENSOR>
-__device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
-                               unsigned char *__restrict__ rec_out, float *__restrict__ dbg,
-                               int32_t *status)
+// Step 1 of the quantiser on the block held in X: the Hadamard rotation
+// along the channels (blockdiag(H_HB) / sqrt(HB); HB = 0 leaves X as it is).
+// All D threads of the CTA must call this.
+template <int D, int HB>
+__device__ __forceinline__ void rotate_block(float2 (&X)[4][16], QuantSmem<D> &sm)
 {
-    constexpr int W = D / 32;
-    using R = Record<D>;
     const int j = threadIdx.x >> 5, l = threadIdx.x & 31;
-
-    // ---- 1. Hadamard rotation along the channels --------------------------
+    (void)j; (void)l;
     if constexpr (HB >= 32) {
 #pragma unroll
         for (int r = 0; r < 4; ++r) fwht32_regs(X[r]);
@@ -143,6 +138,23 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
 #pragma unroll
             for (int k = 0; k < 16; ++k) X[r][k] = __fmul2_rn(X[r][k], f2(nrm, nrm));
     }
+
+}
+
+// Quantise the block held in X (destroyed) into rec_out (global, 16-byte
+// aligned, Record<D>::kBytes); TENSOR 0 = K code order, 1 = V code order.  dbg: NULL or fp32 [T + D + 2*T*D/32] unrounded
+// r, c, s, m.  All D threads of the CTA must call this.
+template <int D, int HB, int TENSOR>
+__device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
+                               unsigned char *__restrict__ rec_out, float *__restrict__ dbg,
+                               int32_t *status)
+{
+    constexpr int W = D / 32;
+    using R = Record<D>;
+    const int j = threadIdx.x >> 5, l = threadIdx.x & 31;
+
+    // ---- 1. Hadamard rotation along the channels --------------------------
+    rotate_block<D, HB>(X, sm);
 
     // ---- 2. dual-axis variance normalisation ------------------------------
     float2 u[16];  // 1 / c for this thread's 32 channels

@@ -32,7 +32,7 @@ KVARN_BF16 = 1
 EXPORTED = (
     "kvarn_record_bytes", "kvarn_cache_bytes", "kvarn_decode_workspace_bytes", "kvarn_quantize_blocks",
     "kvarn_append_token", "kvarn_decode_attention", "kvarn_dequantize", "kvarn_strerror",
-    "kvarn_decode_attention_noalloc",
+    "kvarn_decode_attention_noalloc", "kvarn_token_errors",
 )
 
 
@@ -76,6 +76,7 @@ def lib() -> ctypes.CDLL:
         L.kvarn_decode_attention.argtypes = [P(kvarn_config), V, I, F, P(kvarn_cache), I, V, V, S, V]
         L.kvarn_dequantize.argtypes = [P(kvarn_config), P(kvarn_cache), I, I, I, V, V, V]
         L.kvarn_decode_attention_noalloc.argtypes = [P(kvarn_config), V, I, F, P(kvarn_cache), I, V, V]
+        L.kvarn_token_errors.argtypes = [P(kvarn_config), V, V, I, I, P(kvarn_cache), V, V, V]
         L.kvarn_strerror.argtypes = [I]
         L.kvarn_strerror.restype = ctypes.c_char_p
         for name in ("kvarn_quantize_blocks", "kvarn_append_token", "kvarn_decode_attention", "kvarn_dequantize",
@@ -247,6 +248,18 @@ def decode_attention_noalloc(cfg: Config, q, cache: KVCache, max_tokens: int, ou
                                                 ctypes.byref(cs), int(max_tokens), _ptr(out), _stream(stream)),
            "kvarn_decode_attention_noalloc")
     return out
+
+
+def token_errors(cfg: Config, k, v, cache: KVCache, first_block: int = 0, stream=None):
+    """kvarn_token_errors -> (err_k, err_v) fp32 [S, Hkv, T_total, 2]: per token (|‖x^‖/‖x‖ - 1|, 1 - cos)
+    of the records from first_block on against the original rows k, v [S, Hkv, T_total, D]."""
+    n = k.shape[2]
+    ek = torch.empty(k.shape[0], k.shape[1], n, 2, dtype=torch.float32, device=k.device)
+    ev = torch.empty_like(ek)
+    c, cs = cfg.c(), cache.struct()
+    _check(lib().kvarn_token_errors(ctypes.byref(c), _ptr(k), _ptr(v), int(n), int(first_block), ctypes.byref(cs),
+                                    _ptr(ek), _ptr(ev), _stream(stream)), "kvarn_token_errors")
+    return ek, ev
 
 
 def dequantize(cfg: Config, cache: KVCache, first_block: int, num_blocks: int, rotated: bool = False, stream=None):

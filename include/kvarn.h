@@ -201,6 +201,27 @@ KVARN_API int kvarn_decode_attention(const kvarn_config *cfg, const void *q, int
                            float *out, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Quantisation error of stored blocks, per token, split into magnitude and
+ * direction (article on KVarN, "The Problem": the errors that compound in
+ * K are those of the token magnitudes, not of the directions; "How It
+ * Works": the dual scaling is there to cut the magnitude part).  Compares
+ * the original rows
+ *   k, v  [num_seqs][num_kv_heads][num_tokens][D] in cfg->dtype (the rows
+ *         kvarn_quantize_blocks was given), num_tokens a multiple of T,
+ * with records first_block .. first_block + num_tokens/T - 1, and writes
+ *   err_k, err_v [num_seqs][num_kv_heads][num_tokens][2] fp32:
+ *   (|norm(x^)/norm(x) - 1|, 1 - cos(x^, x)) per token; a zero row gives (0, 0).
+ * Both quantities are invariant under the rotation, so x is rotated as the
+ * quantiser rotates it and x^ = r c (s code + m) from the stored binary16
+ * scales.  Useful with cfg->hadamard = 0 or cfg->sweeps = 0 to measure what
+ * each stage removes.  Errors: KVARN_EINVAL for a ragged num_tokens, a block
+ * range beyond max_blocks, or a NULL / unaligned pointer.
+ */
+KVARN_API int kvarn_token_errors(const kvarn_config *cfg, const void *k, const void *v, int num_tokens,
+                                 int first_block, const kvarn_cache *cache, float *err_k, float *err_v,
+                                 void *stream);
+
+/*
  * Dequantise records first_block .. first_block+num_blocks-1 of every
  * (sequence, kv head) into fp32 k_out / v_out
  * [num_seqs][num_kv_heads][num_blocks*T][D]; rotated != 0 keeps the rotated

@@ -165,6 +165,29 @@ def dequantize_record(rec, T: int, D: int, hb: int, rotated: bool = False, layou
     return out
 
 
+# ------------------------------------------------------ error decomposition
+def magnitude_direction_errors(x, xhat) -> np.ndarray:
+    """Per row of x and its reconstruction xhat (..., D): (|norm(xhat)/norm(x) - 1|, 1 - cos(xhat, x)) in fp64.
+
+    The split the KVarN article draws ("The Problem"; "How It Works"): error in a token's magnitude versus error
+    in its direction.  A zero row of x gives (0, 0); a zero xhat of a nonzero x gives (1, 1).
+    """
+    x = _f64(x)
+    xhat = _f64(xhat)
+    nx = np.sqrt(np.sum(x * x, axis=-1))
+    ny = np.sqrt(np.sum(xhat * xhat, axis=-1))
+    dot = np.sum(x * xhat, axis=-1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        mag = np.where(nx > 0, np.abs(ny / nx - 1.0), 0.0)
+        dirr = np.where(nx > 0, np.where(ny > 0, 1.0 - dot / (nx * ny), 1.0), 0.0)
+    return np.stack([mag, dirr], axis=-1)
+
+
+def record_token_errors(x, rec, T: int, D: int, hb: int, layout: int = NATURAL) -> np.ndarray:
+    """(T, 2) magnitude / direction errors of the T original rows x against their record (original basis)."""
+    return magnitude_direction_errors(x, dequantize_record(rec, T, D, hb, False, layout))
+
+
 # ---------------------------------------------------------------- attention
 def attention(q, K, V, scale: float) -> np.ndarray:
     """q (Hq, D); K, V (Hkv, L, D) -> out (Hq, D) by explicit softmax in fp64."""

@@ -351,3 +351,55 @@ def test_end_to_end_gpu_quantize_and_decode_vs_oracle():
     ref = _oracle_decode(to_f64(q), krec, vrec, to_f64(ocache.k_tail.cpu()), to_f64(ocache.v_tail.cpu()), L, 128,
                          1 / math.sqrt(D))
     assert np.max(np.abs(out - ref)) <= DECODE_ATOL
+
+
+def test_hadamard_absorbed_mode_on_gpu():
+    """Rotation folded into the inputs: hadamard 0 on K, V, q rotated beforehand (fp32) gives the oracle's
+    hadamard-0 result on those inputs, and, rotated back, the standard mode's output."""
+    S, H, Hq, D, L = 2, 2, 8, 128, 3 * 128 + 41
+    k, v = _inputs(S, H, D, L, torch.float32, 4, 0.5, None, 77)
+    q = synth.queries(78, S, Hq, D, dtype=torch.float32)
+    kr = torch.from_numpy(oracle.rotate(to_f64(k), D)).float()
+    vr = torch.from_numpy(oracle.rotate(to_f64(v), D)).float()
+    qr = torch.from_numpy(oracle.rotate(to_f64(q), D)).float()
+    outs = {}
+    for name, (kk, vv, qq, hb) in {"std": (k, v, q, D), "abs": (kr, vr, qr, 0)}.items():
+        cfg = _cfg(S, H, D, 4, torch.float32, hb)
+        cache = kvarn.KVCache(cfg)
+        kvarn.quantize_blocks(cfg, kk.to(DEV), vv.to(DEV), cache)
+        outs[name] = kvarn.decode_attention(cfg, qq.to(DEV), cache, max_tokens=L).cpu().numpy()
+        assert int(cache.status.item()) == 0
+    # parity of the absorbed mode itself: the oracle with hadamard 0 on the same fp32 inputs
+    ocfg = _cfg(S, H, D, 4, torch.float32, 0)
+    _, krec, vrec = _oracle_cache(ocfg, kr, vr, L, 0)
+    nb = L // 128
+    ktail = np.zeros((S, H, 128, D)); vtail = np.zeros((S, H, 128, D))
+    ktail[:, :, :L - nb * 128] = to_f64(kr[:, :, nb * 128:])
+    vtail[:, :, :L - nb * 128] = to_f64(vr[:, :, nb * 128:])
+    ref = _oracle_decode(to_f64(qr), krec, vrec, ktail, vtail, L, 0, 1 / math.sqrt(D))
+    assert np.max(np.abs(outs["abs"] - ref)) <= DECODE_ATOL
+    # rotated back, the standard mode's output
+    back = oracle.rotate(outs["abs"].astype(np.float64), D)
+    assert np.max(np.abs(back - outs["std"])) <= DECODE_ATOL
+
+
+@pytest.mark.parametrize("D,hb,sweeps,dtype", [(128, 128, 4, torch.bfloat16), (128, 0, 4, torch.bfloat16),
+                                               (128, 128, 0, torch.bfloat16), (128, 0, 0, torch.bfloat16),
+                                               (96, 32, 4, torch.float32), (64, 64, 1, torch.float32)])
+def test_token_errors_match_oracle(D, hb, sweeps, dtype):
+    """Per-token magnitude / direction errors on the GPU against the oracle's, on the records the GPU wrote."""
+    S, H, T = 2, 2, 256
+    k, v = _inputs(S, H, D, T, dtype, 4, 0.5, (31, 32, 63, 64) if D == 96 else None, 60 + D + hb + sweeps)
+    cfg = _cfg(S, H, D, 2, dtype, hb, sweeps)
+    cache = kvarn.KVCache(cfg)
+    kd, vd = k.to(DEV), v.to(DEV)
+    kvarn.quantize_blocks(cfg, kd, vd, cache)
+    ek, ev = kvarn.token_errors(cfg, kd, vd, cache)
+    torch.cuda.synchronize()
+    for x, recs, err, lay in ((k, cache.k_records, ek, oracle.K_ORDER), (v, cache.v_records, ev, oracle.V_ORDER)):
+        xs, rs, es = to_f64(x), recs.cpu().numpy(), err.cpu().numpy()
+        for s in range(S):
+            for h in range(H):
+                for b in range(2):
+                    ref = oracle.record_token_errors(xs[s, h, b * 128:(b + 1) * 128], rs[s, h, b], 128, D, hb, lay)
+                    np.testing.assert_allclose(es[s, h, b * 128:(b + 1) * 128], ref, rtol=1e-4, atol=2e-5)

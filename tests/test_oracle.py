@@ -332,3 +332,73 @@ def test_quantize_many_matches_single_blocks():
     kd = k.double().numpy().reshape(4, 128, 64)
     for u in range(4):
         np.testing.assert_array_equal(recs[u], oracle.pack_record(oracle.quantize_block(kd[u], 64, 4)))
+
+
+def test_hadamard_absorbed_mode_identity():
+    """Rotation folded into the inputs (hadamard 0 on pre-rotated K, V, q) is the same encoding, and its output is
+    the rotated output of the standard mode (the rotation is orthogonal and its own inverse)."""
+    rng = np.random.default_rng(31)
+    T, D, Hkv, Hq, n = 8, 64, 1, 2, 19  # two 8-token blocks and a 3-token tail
+    Kx = rng.standard_normal((Hkv, 24, D)) * np.exp(rng.standard_normal(D))
+    Vx = rng.standard_normal((Hkv, 24, D))
+    q = rng.standard_normal((Hq, D))
+    Kr, Vr, qr = oracle.rotate(Kx, D), oracle.rotate(Vx, D), oracle.rotate(q, D)
+    nb = n // T
+    rb = oracle.record_bytes(T, D)
+    recs = {}
+    for name, X, hb in (("std", (Kx, Vx), D), ("abs", (Kr, Vr), 0)):
+        kr = np.zeros((Hkv, nb, rb), dtype=np.uint8)
+        vr = np.zeros_like(kr)
+        for b in range(nb):
+            kr[0, b] = oracle.pack_record(oracle.quantize_block(X[0][0, b * T:(b + 1) * T], hb, 4))
+            vr[0, b] = oracle.pack_record(oracle.quantize_block(X[1][0, b * T:(b + 1) * T], hb, 4))
+        recs[name] = (kr, vr)
+    # the rotation inside the quantiser equals the rotation done beforehand: identical records
+    np.testing.assert_array_equal(recs["std"][0], recs["abs"][0])
+    np.testing.assert_array_equal(recs["std"][1], recs["abs"][1])
+    tail = lambda X: np.concatenate([X[:, nb * T:n], np.zeros((Hkv, T - (n - nb * T), D))], axis=1)
+    out_std = oracle.decode_from_cache(q, *recs["std"], tail(Kx), tail(Vx), n, T, D, 1 / 8)
+    out_abs = oracle.decode_from_cache(qr, *recs["abs"], tail(Kr), tail(Vr), n, T, 0, 1 / 8)
+    np.testing.assert_allclose(oracle.rotate(out_abs, D), out_std, rtol=0, atol=1e-12)
+
+
+def test_error_split_closed_forms():
+    """Magnitude / direction split: a scaled copy has only a magnitude error, an orthogonal one only a direction
+    error of 1, and a rotation of both rows changes neither."""
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((5, 64))
+    a = np.array([0.5, 1.0, 1.25, 2.0, 3.0])
+    e = oracle.magnitude_direction_errors(x, x * a[:, None])
+    np.testing.assert_allclose(e[:, 0], np.abs(a - 1), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(e[:, 1], 0.0, rtol=0, atol=1e-14)
+    y = rng.standard_normal((5, 64))
+    y -= (np.sum(x * y, axis=1) / np.sum(x * x, axis=1))[:, None] * x  # orthogonal to x
+    e = oracle.magnitude_direction_errors(x, y)
+    np.testing.assert_allclose(e[:, 1], 1.0, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(e[:, 0], np.abs(np.linalg.norm(y, axis=1) / np.linalg.norm(x, axis=1) - 1),
+                               rtol=1e-13)
+    z = x + 0.1 * rng.standard_normal((5, 64))
+    np.testing.assert_allclose(oracle.magnitude_direction_errors(oracle.rotate(x, 64), oracle.rotate(z, 64)),
+                               oracle.magnitude_direction_errors(x, z), rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(oracle.magnitude_direction_errors(np.zeros((1, 8)), np.ones((1, 8))), [[0, 0]])
+
+
+def test_record_errors_vanish_on_the_grid_and_grow_without_normalisation():
+    """Values on the 2-bit grid reconstruct exactly (zero error); on the synthetic K the two-stage encoding
+    (rotation + normalisation) leaves a smaller mean magnitude error than plain group RTN."""
+    rng = np.random.default_rng(5)
+    T, D = 128, 64
+    m = rng.integers(-64, 64, size=(T, 2)) / 16.0
+    s = rng.integers(1, 32, size=(T, 2)) / 32.0
+    k = rng.integers(0, 4, size=(T, D))
+    k[:, 0], k[:, 1], k[:, 32], k[:, 33] = 0, 3, 0, 3
+    X = m.repeat(32, axis=1) + k * s.repeat(32, axis=1)
+    rec = oracle.pack_record(oracle.quantize_block(X, hb=0, sweeps=0))
+    np.testing.assert_allclose(oracle.record_token_errors(X, rec, T, D, 0), 0.0, rtol=0, atol=1e-14)
+    K, _ = _config0_k(3)
+    K = K[:128]
+    err = {}
+    for name, hb, sw in (("kvarn", 64, 4), ("rtn", 0, 0)):
+        rec = oracle.pack_record(oracle.quantize_block(K, hb, sw))
+        err[name] = oracle.record_token_errors(K, rec, T, D, hb).mean(axis=0)
+    assert err["kvarn"][0] < err["rtn"][0]
