@@ -64,6 +64,14 @@ struct alignas(128) DecWarpSmem {
     unsigned long long mbar[2];               // K record, V record
 };
 
+// Channel groups a lane's P V rows cover (its copy's groups): the lane keeps
+// the running output of those groups' n-tiles only.
+template <int D, int GRP>
+__host__ __device__ constexpr int dec_sets()
+{
+    return (D / kGroup + 8 / GRP - 1) / (8 / GRP);
+}
+
 // Warps per CTA: up to 12, as many as fit in 227 KB of shared memory.
 template <int D, int GRP>
 __host__ __device__ constexpr int dec_warps()
@@ -256,6 +264,15 @@ constexpr int kTailSlots = 3;
 // Marker of a unit whose merge the completing warp left to its CTA.
 constexpr uint32_t kMergeFlag = 0x80000000u;
 
+// 2^x for x <= 0 (softmax weights): the hardware approximation, subnormal
+// results flushed to zero (relative error about 2^-22).
+__device__ __forceinline__ float exp2_ftz(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // fp32 pair -> the fp16 pair of its high part (hl = 0) or of its remainder (hl = 1).
 __device__ __forceinline__ uint32_t hilo_part(float x, float y, bool hl)
 {
@@ -314,7 +331,7 @@ __device__ __forceinline__ void convert_k_scales(const unsigned char *rec, float
 template <int D, int GRP, typename Tin>
 __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, const unsigned char *vbase, int b0,
                            int b1, uint32_t &kph, uint32_t &vph, float (&m_run)[(GRP + 3) / 4],
-                           float (&l_run)[(GRP + 3) / 4], float2 (&orun)[D / 8])
+                           float (&l_run)[(GRP + 3) / 4], float2 (&orun)[dec_sets<D, GRP>()][kGroup / 8])
 {
     using R = Record<D>;
     constexpr int NG = D / kGroup;          // channel groups
@@ -470,12 +487,12 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
             mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 8));
             mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 16));
             const float mnew = fmaxf(m_run[j], mb);
-            alpha[j] = exp2f(m_run[j] - mnew);
+            alpha[j] = exp2_ftz(m_run[j] - mnew);
             float ls = 0.f;
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                sc[j][u][0] = exp2f(sc[j][u][0] - mnew);
-                sc[j][u][1] = exp2f(sc[j][u][1] - mnew);
+                sc[j][u][0] = exp2_ftz(sc[j][u][0] - mnew);
+                sc[j][u][1] = exp2_ftz(sc[j][u][1] - mnew);
                 ls += sc[j][u][0] + sc[j][u][1];
             }
             ls += __shfl_xor_sync(0xffffffffu, ls, 4);
@@ -552,7 +569,9 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
 
         // ---- P V, one group set at a time
 #pragma unroll
-        for (int i2 = 0; i2 < NNT; ++i2) orun[i2] = __fmul2_rn(orun[i2], f2(alphaV, alphaV));
+        for (int st = 0; st < SETS; ++st)
+#pragma unroll
+            for (int jn = 0; jn < kGroup / 8; ++jn) orun[st][jn] = __fmul2_rn(orun[st][jn], f2(alphaV, alphaV));
 #pragma unroll
         for (int st = 0; st < SETS; ++st) {
             const int g = st * C + copy;
@@ -577,13 +596,14 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
             const float bx = __shfl_sync(0xffffffffu, bpair.x, 4 * h + gsrc / 2);
             const float by = __shfl_sync(0xffffffffu, bpair.y, 4 * h + gsrc / 2);
             const float bias = ((gsrc & 1) ? by : bx) * kTwoM16;
+            // two 8-channel n-tiles at a time: independent MMA chains interleave
 #pragma unroll
-            for (int cc = 0; cc < C; ++cc) {
-                const int gg = st * C + cc;
-                if (gg >= NG) continue;
-                // two 8-channel n-tiles at once: independent MMA chains interleave
+            for (int j4 = 0; j4 < kGroup / 8; j4 += 2) {
+                float mine[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-                for (int j4 = 0; j4 < kGroup / 8; j4 += 2) {
+                for (int cc = 0; cc < C; ++cc) {
+                    const int gg = st * C + cc;
+                    if (gg >= NG) continue;
                     const int nt0 = gg * (kGroup / 8) + j4;
                     CodeWord vw[2][2];
                     float acc4[2][4];
@@ -607,15 +627,20 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
                             mma16816(acc4[jj], Av[ks], bb[0], bb[1]);
                         }
                     }
-                    if (cc == copy) {
+                    // the rows of this lane's copy carry the heads of group gg only when cc == copy
 #pragma unroll
-                        for (int jj = 0; jj < 2; ++jj) {
-                            const int nt = nt0 + jj;
-                            const float2 cv = *reinterpret_cast<const float2 *>(cV + 8 * nt + 2 * tig);
-                            const float2 hs = hilo_sum(acc4[jj]);
-                            const float2 o = f2(hs.x + bias, hs.y + bias);
-                            orun[nt] = __ffma2_rn(o, cv, orun[nt]);
-                        }
+                    for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) mine[jj][i] = cc == copy ? acc4[jj][i] : mine[jj][i];
+                }
+                if (gv) {
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int nt = g * (kGroup / 8) + j4 + jj;
+                        const float2 cv = *reinterpret_cast<const float2 *>(cV + 8 * nt + 2 * tig);
+                        const float2 hs = hilo_sum(mine[jj]);
+                        const float2 o = f2(hs.x + bias, hs.y + bias);
+                        orun[st][j4 + jj] = __ffma2_rn(o, cv, orun[st][j4 + jj]);
                     }
                 }
             }
@@ -941,8 +966,9 @@ decode_kernel(DecodeArgs a, int hb)
 {
     using R = Record<D>;
     constexpr int W = dec_warps<D, GRP>();
-    constexpr int NNT = D / 8;
     constexpr int C = 8 / GRP;
+    constexpr int NG = D / kGroup;
+    constexpr int SETS = dec_sets<D, GRP>();
     constexpr int NTN = (GRP + 3) / 4;
     constexpr int SR = slot_row<D>();
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -987,9 +1013,11 @@ decode_kernel(DecodeArgs a, int hb)
         float m_run[NTN], l_run[NTN];
 #pragma unroll
         for (int j = 0; j < NTN; ++j) { m_run[j] = -INFINITY; l_run[j] = 0.f; }
-        float2 orun[NNT];
+        float2 orun[SETS][kGroup / 8];  // this lane's groups st * C + copy, their four n-tiles
 #pragma unroll
-        for (int j = 0; j < NNT; ++j) orun[j] = f2(0.f, 0.f);
+        for (int st = 0; st < SETS; ++st)
+#pragma unroll
+            for (int jn = 0; jn < kGroup / 8; ++jn) orun[st][jn] = f2(0.f, 0.f);
         if (b0 < b1r && !dead) {
             // rotated query of this GQA group, scaled by softmax scale * log2(e)
             const Tin *qg = static_cast<const Tin *>(a.q) + (size_t)unit * GRP * D;
@@ -1006,7 +1034,9 @@ decode_kernel(DecodeArgs a, int hb)
 #pragma unroll
                 for (int j = 0; j < NTN; ++j) { m_run[j] = -INFINITY; l_run[j] = 0.f; }
 #pragma unroll
-                for (int j = 0; j < NNT; ++j) orun[j] = f2(0.f, 0.f);
+                for (int st = 0; st < SETS; ++st)
+#pragma unroll
+                    for (int jn = 0; jn < kGroup / 8; ++jn) orun[st][jn] = f2(0.f, 0.f);
             }
         }
         // ---- this segment's block partial: (m, l, o_rot) per head
@@ -1021,9 +1051,12 @@ decode_kernel(DecodeArgs a, int hb)
                 }
             float *pp = slot + h * SR;
 #pragma unroll
-            for (int nt = 0; nt < NNT; ++nt) {
-                if ((nt / (kGroup / 8)) % C == copy)
-                    *reinterpret_cast<float2 *>(pp + 4 + 8 * nt + 2 * tig) = orun[nt];
+            for (int st = 0; st < SETS; ++st) {
+                const int g = st * C + copy;
+                if (g < NG)
+#pragma unroll
+                    for (int jn = 0; jn < kGroup / 8; ++jn)
+                        *reinterpret_cast<float2 *>(pp + 4 + 8 * (g * (kGroup / 8) + jn) + 2 * tig) = orun[st][jn];
             }
         }
         if (has_tail) tail_partial<D, GRP, Tin>(a, sm, unit, ntail, a.tail_partials + (size_t)unit * GRP * SR);
