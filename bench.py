@@ -41,7 +41,7 @@ QB_WORKLOAD = "Llama-3-8B-shaped bulk prefill quantise: 32 batch x 32 layers x 8
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one decode launch at context 32705 for this
 # batch, from one ncu capture of `bench.py --profile decode` with the current decode kernel; reset it to None
 # whenever the decode kernel changes until it is captured again.
-DECODE_TRAFFIC_BYTES = 219942400 + 4037888
+DECODE_TRAFFIC_BYTES = None  # decode kernel changed since the last capture
 
 
 def _peaks():
@@ -252,9 +252,10 @@ def run_kvarn(args, world, rank, local):
     if not args.skip_quant:
         quant = run_bulk_quant(args, dev, seed, peak)
     ablation = None if args.skip_ablation or rank != 0 else run_ablation(dev)
+    multi = None if args.skip_ablation or rank != 0 else run_multi_query(dev, peak)
 
     return dict(value=value, ms_step=ms_step, clocks=clk, dec_avg_ms=dec_avg_ms, dbytes=dbytes, achieved=achieved,
-                peak=peak, peak_kind=peak_kind, e2e_value=e2e_value, h2d=h2d, d2h=d2h, quant=quant, ablation=ablation,
+                peak=peak, peak_kind=peak_kind, e2e_value=e2e_value, h2d=h2d, d2h=d2h, quant=quant, ablation=ablation, multi=multi,
                 launches=args.steps * T_BLK * LAYERS * 2)
 
 
@@ -387,6 +388,42 @@ def run_ablation(dev):
     return out
 
 
+# ------------------------------------------------------------------- several query tokens at once
+def run_multi_query(dev, peak):
+    """One Qwen3-4B-shaped layer at 32705 cached tokens: decode of the last token alone versus the last two
+    tokens at once (speculative verification); 2 queries x GQA 4 fill the 8 rows of the tensor-core tiles."""
+    from bit_kv_cache_token_b200 import kvarn, synth
+    cfg = kvarn.Config(S, HKV, D, max_blocks=32768 // T_BLK, hadamard=D, dtype=kvarn.KVARN_BF16)
+    caches = []
+    for layer in range(4):  # distinct layers so that L2 cannot hold the working set
+        k, v = synth.layer_kv(11, layer, S, HKV, CTX0 + 65, D, device=dev)
+        c = kvarn.KVCache(cfg, device=dev)
+        kvarn.quantize_blocks(cfg, k, v, c)
+        caches.append(c)
+        del k, v
+    res = {}
+    for Q in (1, 2):
+        q = synth.queries(12, S * Q, HQ, D, device=dev).reshape(S, Q, HQ, D)
+        ws = kvarn.decode_workspace(cfg, Q * HQ, dev)
+        out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+        for c in caches:
+            kvarn.decode_attention_multi(cfg, q, c, max_tokens=32768, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
+        e0.record()
+        for _ in range(reps):
+            for c in caches:
+                kvarn.decode_attention_multi(cfg, q, c, max_tokens=32768, out=out, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (reps * len(caches))
+        gbs = decode_bytes(CTX0 + 65) / (us * 1e-6) / 1e9
+        res[f"q{Q}"] = {"us_per_launch": us, "us_per_query_token": us / Q, "gbs": gbs, "frac": gbs / peak}
+    res["workload"] = "Qwen3-4B-shaped layer, batch 8, 32705 cached tokens; the last 1 or 2 tokens as queries"
+    return res
+
+
 # ------------------------------------------------------------------- small profiling cases
 def run_profile_case(case: str):
     """Small cases for ncu captures: 3 launches of one kernel on inputs larger than L2.
@@ -432,7 +469,7 @@ def main():
     ap.add_argument("--skip-quant", action="store_true", help="skip the bulk quantise measurement")
     ap.add_argument("--small", action="store_true", help="reduced bulk quantise size (quick checks)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--skip-ablation", action="store_true", help="skip the rotation / normalisation ablation")
+    ap.add_argument("--skip-ablation", action="store_true", help="skip the ablation and multi-query measurements")
     ap.add_argument("--profile", choices=["decode", "quantize", "append"], default=None,
                     help="run a small case of one kernel for ncu and exit")
     args = ap.parse_args()
@@ -492,6 +529,8 @@ def main():
                                 "algorithmic_bytes": q["bytes"], "peak": r["peak"], "status": q["status"]}
         if r["ablation"]:
             line["ablation"] = r["ablation"]
+        if r["multi"]:
+            line["multi_query_decode"] = r["multi"]
         if cpu:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)

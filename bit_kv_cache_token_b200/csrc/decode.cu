@@ -249,6 +249,18 @@ __device__ __forceinline__ long long part_owner(long long i, long long total, lo
     return ((i + 1) * nw + total - 1) / total - 1;
 }
 
+// Element offset of row v (query v / heads_per_kv, head v % heads_per_kv) of
+// unit (sequence s, kv head hk) in q and out, laid out [S][num_queries][Hq][D].
+template <int D, int GRP, bool MQ>
+__device__ __forceinline__ size_t qo_row(const DecodeArgs &a, int unit, int v)
+{
+    if constexpr (!MQ) return ((size_t)unit * GRP + v) * D;  // one query: [S][Hq][D]
+    const int s = unit / a.num_kv_heads, hk = unit % a.num_kv_heads;
+    const int qi = v / a.heads_per_kv, h = v % a.heads_per_kv;
+    const int hq = a.num_kv_heads * a.heads_per_kv;
+    return (((size_t)s * a.num_queries + qi) * hq + (size_t)hk * a.heads_per_kv + h) * D;
+}
+
 // Slot layout of a partial: per head [m, l, pad, pad, o[D]] (16-byte aligned rows).
 template <int D>
 __host__ __device__ constexpr int slot_row() { return D + 4; }
@@ -328,10 +340,11 @@ __device__ __forceinline__ void convert_k_scales(const unsigned char *rec, float
 // head.  P V keeps the head-rows layout (A = p r s rows, B = V codes), whose
 // lanes get their probabilities from the score lanes by shuffles; orun is
 // in that layout (head gl % GRP).
-template <int D, int GRP, typename Tin>
+template <int D, int GRP, typename Tin, bool MQ>
 __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, const unsigned char *vbase, int b0,
                            int b1, uint32_t &kph, uint32_t &vph, float (&m_run)[(GRP + 3) / 4],
-                           float (&l_run)[(GRP + 3) / 4], float2 (&orun)[dec_sets<D, GRP>()][kGroup / 8])
+                           float (&l_run)[(GRP + 3) / 4], float2 (&orun)[dec_sets<D, GRP>()][kGroup / 8],
+                           int blim0, int hpk)
 {
     using R = Record<D>;
     constexpr int NG = D / kGroup;          // channel groups
@@ -364,6 +377,9 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
         const unsigned char *krec = sm.rec[0];
         const unsigned char *vrec = sm.rec[1];
         float *scr = sm.scr;
+        // several queries: row v sees positions <= blim0 + v / hpk; only a block
+        // reaching past blim0 needs the mask
+        const bool masked = b * kBlockTokens + kBlockTokens - 1 > blim0;
 
         // ---- K scales: srK[t][4] = s r 2^16, rK[t], cK[d]
         float *srK = scr, *rK = scr + 4 * kBlockTokens, *cK = scr + 5 * kBlockTokens;
@@ -476,6 +492,19 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
             }
         }
 
+        if (MQ && masked) {  // only the last block, when several queries end inside it
+#pragma unroll
+            for (int j = 0; j < NTN; ++j) {
+                const int lim = blim0 + (4 * j + tig) / hpk;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int pa = b * kBlockTokens + 16 * u + gl;
+                    if (pa > lim) sc[j][u][0] = -INFINITY;
+                    if (pa + 8 > lim) sc[j][u][1] = -INFINITY;
+                }
+            }
+        }
+
         // ---- online softmax (base 2; the scale carries log2(e)), per head 4j + tig
         float alpha[NTN];
 #pragma unroll
@@ -487,12 +516,14 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
             mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 8));
             mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 16));
             const float mnew = fmaxf(m_run[j], mb);
-            alpha[j] = exp2_ftz(m_run[j] - mnew);
+            // several queries: a row may see nothing yet, and its weights must stay 0
+            const float msub = (MQ && mnew == -INFINITY) ? 0.f : mnew;
+            alpha[j] = exp2_ftz(m_run[j] - msub);
             float ls = 0.f;
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                sc[j][u][0] = exp2_ftz(sc[j][u][0] - mnew);
-                sc[j][u][1] = exp2_ftz(sc[j][u][1] - mnew);
+                sc[j][u][0] = exp2_ftz(sc[j][u][0] - msub);
+                sc[j][u][1] = exp2_ftz(sc[j][u][1] - msub);
                 ls += sc[j][u][0] + sc[j][u][1];
             }
             ls += __shfl_xor_sync(0xffffffffu, ls, 4);
@@ -658,8 +689,8 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
 // tail partial (m, l, o per head, unrotated basis) to dst.  The tail is at
 // most 127 tokens and its cost is latency: every loop keeps a whole row (K)
 // or 16 rows (V) of loads in flight.
-template <int D, int GRP, typename Tin>
-__device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int unit, int ntail, float *dst)
+template <int D, int GRP, typename Tin, bool MQ>
+__device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int unit, int ntail, int tlim0, float *dst)
 {
     constexpr int SR = slot_row<D>();
     constexpr int VB = 16;  // V rows per batch of loads
@@ -667,8 +698,16 @@ __device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int u
     float *ps = reinterpret_cast<float *>(sm.rec[0]);  // [128][GRP] scores, then weights
     float *qt = ps + kBlockTokens * GRP;               // [GRP][D] query, scaled (uniform reads: broadcasts)
     static_assert(sizeof(float) * (kBlockTokens * GRP + GRP * D) <= sizeof(sm.rec), "tail scratch");
-    const Tin *qg = static_cast<const Tin *>(a.q) + (size_t)unit * GRP * D;
-    for (int i = lane; i < GRP * D; i += 32) qt[i] = In<Tin>::load1(qg + i) * a.scale_log2;
+    if constexpr (MQ) {
+#pragma unroll
+        for (int v = 0; v < GRP; ++v) {
+            const Tin *qv = static_cast<const Tin *>(a.q) + qo_row<D, GRP, MQ>(a, unit, v);
+            for (int d = lane; d < D; d += 32) qt[v * D + d] = In<Tin>::load1(qv + d) * a.scale_log2;
+        }
+    } else {
+        const Tin *qg = static_cast<const Tin *>(a.q) + (size_t)unit * GRP * D;
+        for (int i = lane; i < GRP * D; i += 32) qt[i] = In<Tin>::load1(qg + i) * a.scale_log2;
+    }
     __syncwarp();
     // scores: lanes over tokens, a row's loads issued together
     const Tin *kt = static_cast<const Tin *>(a.k_tail) + (size_t)unit * kBlockTokens * D;
@@ -697,8 +736,10 @@ __device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int u
                     acc[hh] = fmaf(qv.w, kv[c4 + 3], acc[hh]);
                 }
             }
+            // several queries: row hh sees tail tokens t <= tlim0 + hh / heads_per_kv
 #pragma unroll
-            for (int hh = 0; hh < GRP; ++hh) ps[t * GRP + hh] = acc[hh];
+            for (int hh = 0; hh < GRP; ++hh)
+                ps[t * GRP + hh] = (!MQ || t <= tlim0 + hh / a.heads_per_kv) ? acc[hh] : -INFINITY;
         }
     }
     __syncwarp();
@@ -719,7 +760,7 @@ __device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int u
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int t = lane + 32 * j;
-            const float p = t < ntail ? exp2f(sv[j] - mx) : 0.f;
+            const float p = (t < ntail && (!MQ || sv[j] > -INFINITY)) ? exp2f(sv[j] - mx) : 0.f;
             if (t < ntail) ps[t * GRP + hh] = p;
             sum += p;
         }
@@ -768,7 +809,7 @@ __device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int u
 // Merge of one unit by a single warp (few partials): block partials from the
 // slots of warps [wf, wl] (empty ranges skipped), the tail partial, the
 // un-rotation, the output.  Uses the warp's record buffers as scratch.
-template <int D, int GRP>
+template <int D, int GRP, bool MQ>
 __device__ void warp_merge(const DecodeArgs &a, int hb, DecWarpSmem<D, GRP> &sm, int unit, long long wf, long long wl,
                            long long total, long long nw)
 {
@@ -816,8 +857,16 @@ __device__ void warp_merge(const DecodeArgs &a, int hb, DecWarpSmem<D, GRP> &sm,
     }
     __syncwarp();
     warp_fwht<D>(obuf, GRP, hb);
-    float *out = a.out + (size_t)unit * GRP * D;
-    for (int i = lane; i < GRP * D; i += 32) out[i] = obuf[i] + otl[i];
+    if constexpr (MQ) {
+#pragma unroll
+        for (int v = 0; v < GRP; ++v) {
+            float *ov = a.out + qo_row<D, GRP, MQ>(a, unit, v);
+            for (int d = lane; d < D; d += 32) ov[d] = obuf[v * D + d] + otl[v * D + d];
+        }
+    } else {
+        float *out = a.out + (size_t)unit * GRP * D;
+        for (int i = lane; i < GRP * D; i += 32) out[i] = obuf[i] + otl[i];
+    }
     __syncwarp();
 }
 
@@ -825,7 +874,7 @@ __device__ void warp_merge(const DecodeArgs &a, int hb, DecWarpSmem<D, GRP> &sm,
 // of the CTA calls it with the same arguments; the whole dynamic shared
 // memory is scratch.  A slot of a warp whose range is empty was never
 // written: it is neither read nor weighted.
-template <int D, int GRP>
+template <int D, int GRP, bool MQ>
 __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int unit, long long wf, long long wl,
                           long long total, long long nw)
 {
@@ -943,8 +992,18 @@ __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int 
     __syncthreads();
     if (warp < GRP) warp_fwht<D>(obuf + warp * D, 1, hb);
     __syncthreads();
-    float *out = a.out + (size_t)unit * GRP * D;
-    for (int i = tid; i < GRP * D; i += NT) out[i] = obuf[i] + otl[i];
+    if constexpr (MQ) {
+        if (tid < GRP * (D / 4)) {  // a float4 of one row per thread
+            const int v = tid / (D / 4), d4 = tid % (D / 4);
+            const float4 x = *reinterpret_cast<const float4 *>(obuf + v * D + 4 * d4);
+            const float4 y = *reinterpret_cast<const float4 *>(otl + v * D + 4 * d4);
+            *reinterpret_cast<float4 *>(a.out + qo_row<D, GRP, MQ>(a, unit, v) + 4 * d4) =
+                make_float4(x.x + y.x, x.y + y.y, x.z + y.z, x.w + y.w);
+        }
+    } else {
+        float *out = a.out + (size_t)unit * GRP * D;
+        for (int i = tid; i < GRP * D; i += NT) out[i] = obuf[i] + otl[i];
+    }
     __syncthreads();  // the scratch is free again
 }
 
@@ -960,7 +1019,7 @@ __host__ __device__ constexpr int cta_merge_max()
     return (int)((sizeof(DecWarpSmem<D, GRP>) * W - fixed) / (GRP * 12));
 }
 
-template <int D, int GRP, typename Tin>
+template <int D, int GRP, typename Tin, bool MQ>
 __global__ void __launch_bounds__(dec_warps<D, GRP>() * 32, 1)
 decode_kernel(DecodeArgs a, int hb)
 {
@@ -1020,15 +1079,24 @@ decode_kernel(DecodeArgs a, int hb)
             for (int jn = 0; jn < kGroup / 8; ++jn) orun[st][jn] = f2(0.f, 0.f);
         if (b0 < b1r && !dead) {
             // rotated query of this GQA group, scaled by softmax scale * log2(e)
-            const Tin *qg = static_cast<const Tin *>(a.q) + (size_t)unit * GRP * D;
-            for (int j = lane; j < GRP * D; j += 32) (&sm.qbuf[0][0])[j] = In<Tin>::load1(qg + j) * a.scale_log2;
+            if constexpr (MQ) {
+#pragma unroll
+                for (int v = 0; v < GRP; ++v) {
+                    const Tin *qv = static_cast<const Tin *>(a.q) + qo_row<D, GRP, MQ>(a, unit, v);
+                    for (int d = lane; d < D; d += 32) sm.qbuf[v][d] = In<Tin>::load1(qv + d) * a.scale_log2;
+                }
+            } else {
+                const Tin *qg = static_cast<const Tin *>(a.q) + (size_t)unit * GRP * D;
+                for (int j = lane; j < GRP * D; j += 32) (&sm.qbuf[0][0])[j] = In<Tin>::load1(qg + j) * a.scale_log2;
+            }
             __syncwarp();
             warp_fwht<D>(&sm.qbuf[0][0], GRP, hb);
             const unsigned char *kbase =
                 static_cast<const unsigned char *>(a.k_records) + (size_t)unit * a.max_blocks * R::kBytes;
             const unsigned char *vbase =
                 static_cast<const unsigned char *>(a.v_records) + (size_t)unit * a.max_blocks * R::kBytes;
-            if (!run_blocks<D, GRP, Tin>(sm, kbase, vbase, b0, b1r, kph, vph, m_run, l_run, orun)) {
+            if (!run_blocks<D, GRP, Tin, MQ>(sm, kbase, vbase, b0, b1r, kph, vph, m_run, l_run, orun, n - a.num_queries,
+                                         a.heads_per_kv)) {
                 dead = true;
                 if (lane == 0) status_or(a.status, KVARN_STATUS_TIMEOUT);
 #pragma unroll
@@ -1059,7 +1127,9 @@ decode_kernel(DecodeArgs a, int hb)
                         *reinterpret_cast<float2 *>(pp + 4 + 8 * (g * (kGroup / 8) + jn) + 2 * tig) = orun[st][jn];
             }
         }
-        if (has_tail) tail_partial<D, GRP, Tin>(a, sm, unit, ntail, a.tail_partials + (size_t)unit * GRP * SR);
+        if (has_tail)
+            tail_partial<D, GRP, Tin, MQ>(a, sm, unit, ntail, n - a.num_queries - nblk * kBlockTokens,
+                                      a.tail_partials + (size_t)unit * GRP * SR);
 
         // ---- arrival: this segment's items are done
         __syncwarp();
@@ -1073,7 +1143,7 @@ decode_kernel(DecodeArgs a, int hb)
             const long long wf = part_owner(ibase, total, nw), wl = part_owner(ibase + per_unit - 1, total, nw);
             const long long span = wl - wf + 1;
             if (span <= kWarpMergeMax || span > cta_merge_max<D, GRP>()) {
-                warp_merge<D, GRP>(a, hb, sm, unit, wf, wl, total, nw);
+                warp_merge<D, GRP, MQ>(a, hb, sm, unit, wf, wl, total, nw);
                 if (lane == 0) a.tickets[unit] = 0u;
             } else if (lane == 0) {
                 atomicExch(a.tickets + unit, kMergeFlag | blockIdx.x);
@@ -1113,21 +1183,30 @@ decode_kernel(DecodeArgs a, int hb)
         const int unit = merge_list[j];
         const long long ibase = (long long)unit * per_unit;
         const long long wf = part_owner(ibase, total, nw), wl = part_owner(ibase + per_unit - 1, total, nw);
-        cta_merge<D, GRP>(a, hb, smem_raw, unit, wf, wl, total, nw);
+        cta_merge<D, GRP, MQ>(a, hb, smem_raw, unit, wf, wl, total, nw);
         if (threadIdx.x == 0) a.tickets[unit] = 0u;
     }
 }
 
-template <int D, int GRP, typename Tin>
-static cudaError_t launch_dec(const DecodeArgs &a, int hb, int ctas, cudaStream_t st)
+template <int D, int GRP, typename Tin, bool MQ>
+static cudaError_t launch_dec_mq(const DecodeArgs &a, int hb, int ctas, cudaStream_t st)
 {
     constexpr int W = dec_warps<D, GRP>();
     const size_t smem = sizeof(DecWarpSmem<D, GRP>) * W;
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, GRP, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, GRP, Tin, MQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    decode_kernel<D, GRP, Tin><<<ctas, W * 32, smem, st>>>(a, hb);
+    decode_kernel<D, GRP, Tin, MQ><<<ctas, W * 32, smem, st>>>(a, hb);
     return cudaGetLastError();
+}
+
+// One query per sequence (the common case) runs the kernel without the
+// causal masking and row mapping of several queries.
+template <int D, int GRP, typename Tin>
+static cudaError_t launch_dec(const DecodeArgs &a, int hb, int ctas, cudaStream_t st)
+{
+    return a.num_queries > 1 ? launch_dec_mq<D, GRP, Tin, true>(a, hb, ctas, st)
+                             : launch_dec_mq<D, GRP, Tin, false>(a, hb, ctas, st);
 }
 
 template <int D, int GRP>

@@ -144,21 +144,24 @@ int kvarn_append_token(const kvarn_config *cfg, const void *k, const void *v, co
     return cuda_status(run_append(*cfg, a, static_cast<cudaStream_t>(stream)));
 }
 
-int kvarn_decode_attention(const kvarn_config *cfg, const void *q, int num_q_heads, float softmax_scale,
-                           const kvarn_cache *cache, int max_tokens, float *out, void *workspace,
-                           size_t workspace_bytes, void *stream)
+static int decode_impl(const kvarn_config *cfg, const void *q, int num_q_heads, int num_queries,
+                       float softmax_scale, const kvarn_cache *cache, int max_tokens, float *out, void *workspace,
+                       size_t workspace_bytes, void *stream)
 {
     int rc = check_config(cfg);
     if (rc) return rc;
     if ((rc = check_cache(cache, false))) return rc;
     if (!q || !out || !aligned16(q) || !aligned16(out)) return KVARN_EINVAL;
     if (num_q_heads < cfg->num_kv_heads || num_q_heads % cfg->num_kv_heads) return KVARN_EINVAL;
-    const int grp = num_q_heads / cfg->num_kv_heads;
-    if (grp != 1 && grp != 2 && grp != 4 && grp != 8) return KVARN_EUNSUPPORTED;
+    if (num_queries < 1) return KVARN_EINVAL;
+    const int hpk = num_q_heads / cfg->num_kv_heads;
+    if ((long long)hpk * num_queries > 8) return KVARN_EUNSUPPORTED;
+    const int rows = hpk * num_queries;  // rows sharing one kv head
+    if (rows != 1 && rows != 2 && rows != 4 && rows != 8) return KVARN_EUNSUPPORTED;
     if (max_tokens < 0 || (long long)max_tokens > (long long)cfg->max_blocks * cfg->block_tokens + cfg->block_tokens - 1)
         return KVARN_EINVAL;
     if (!(softmax_scale == softmax_scale) || isinf(softmax_scale)) return KVARN_EINVAL;
-    const size_t need = kvarn_decode_workspace_bytes(cfg, num_q_heads);
+    const size_t need = kvarn_decode_workspace_bytes(cfg, num_q_heads * num_queries);
     if (!workspace || !aligned16(workspace) || workspace_bytes < need) return KVARN_EWORKSPACE;
 
     // a persistent grid: one CTA of decode_warps_per_cta warps per SM, the
@@ -173,13 +176,30 @@ int kvarn_decode_attention(const kvarn_config *cfg, const void *q, int num_q_hea
     a.out = out;
     a.tickets = static_cast<uint32_t *>(workspace);
     a.partials = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + ticket_bytes(cfg));
-    a.tail_partials = a.partials + ((size_t)ctas * decode_warps_per_cta(cfg->head_dim, grp) + units) *
-                                       (decode_slot_bytes(cfg->head_dim, grp) / sizeof(float));
+    a.tail_partials = a.partials + ((size_t)ctas * decode_warps_per_cta(cfg->head_dim, rows) + units) *
+                                       (decode_slot_bytes(cfg->head_dim, rows) / sizeof(float));
     const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)cfg->head_dim);
     a.scale_log2 = scale * 1.4426950408889634f;
-    a.num_kv_heads = cfg->num_kv_heads; a.grp = grp; a.max_blocks = cfg->max_blocks;
+    a.num_kv_heads = cfg->num_kv_heads; a.grp = rows; a.max_blocks = cfg->max_blocks;
     a.max_tokens = max_tokens; a.num_units = units;
+    a.num_queries = num_queries; a.heads_per_kv = hpk;
     return cuda_status(run_decode(*cfg, a, ctas, static_cast<cudaStream_t>(stream)));
+}
+
+int kvarn_decode_attention(const kvarn_config *cfg, const void *q, int num_q_heads, float softmax_scale,
+                           const kvarn_cache *cache, int max_tokens, float *out, void *workspace,
+                           size_t workspace_bytes, void *stream)
+{
+    return decode_impl(cfg, q, num_q_heads, 1, softmax_scale, cache, max_tokens, out, workspace, workspace_bytes,
+                       stream);
+}
+
+int kvarn_decode_attention_multi(const kvarn_config *cfg, const void *q, int num_q_heads, int num_queries,
+                                 float softmax_scale, const kvarn_cache *cache, int max_tokens, float *out,
+                                 void *workspace, size_t workspace_bytes, void *stream)
+{
+    return decode_impl(cfg, q, num_q_heads, num_queries, softmax_scale, cache, max_tokens, out, workspace,
+                       workspace_bytes, stream);
 }
 
 int kvarn_token_errors(const kvarn_config *cfg, const void *k, const void *v, int num_tokens, int first_block,

@@ -48,6 +48,11 @@ struct DecodeArgs {
     float scale_log2;           // softmax scale * log2(e)
     int num_kv_heads, grp, max_blocks, max_tokens;
     int num_units;              // S * Hkv
+    // Several query tokens per sequence: grp = num_queries * heads_per_kv rows
+    // share a kv head; row v is query v / heads_per_kv of head v % heads_per_kv.
+    // q and out are [S][num_queries][Hq][D]; query i of a sequence with n
+    // tokens sits at position n - num_queries + i and sees positions <= it.
+    int num_queries, heads_per_kv;
 };
 
 struct ErrorArgs {

@@ -32,7 +32,7 @@ KVARN_BF16 = 1
 EXPORTED = (
     "kvarn_record_bytes", "kvarn_cache_bytes", "kvarn_decode_workspace_bytes", "kvarn_quantize_blocks",
     "kvarn_append_token", "kvarn_decode_attention", "kvarn_dequantize", "kvarn_strerror",
-    "kvarn_decode_attention_noalloc", "kvarn_token_errors",
+    "kvarn_decode_attention_noalloc", "kvarn_token_errors", "kvarn_decode_attention_multi",
 )
 
 
@@ -77,6 +77,7 @@ def lib() -> ctypes.CDLL:
         L.kvarn_dequantize.argtypes = [P(kvarn_config), P(kvarn_cache), I, I, I, V, V, V]
         L.kvarn_decode_attention_noalloc.argtypes = [P(kvarn_config), V, I, F, P(kvarn_cache), I, V, V]
         L.kvarn_token_errors.argtypes = [P(kvarn_config), V, V, I, I, P(kvarn_cache), V, V, V]
+        L.kvarn_decode_attention_multi.argtypes = [P(kvarn_config), V, I, I, F, P(kvarn_cache), I, V, V, S, V]
         L.kvarn_strerror.argtypes = [I]
         L.kvarn_strerror.restype = ctypes.c_char_p
         for name in ("kvarn_quantize_blocks", "kvarn_append_token", "kvarn_decode_attention", "kvarn_dequantize",
@@ -247,6 +248,24 @@ def decode_attention_noalloc(cfg: Config, q, cache: KVCache, max_tokens: int, ou
     _check(lib().kvarn_decode_attention_noalloc(ctypes.byref(c), _ptr(q), int(q.shape[1]), float(softmax_scale),
                                                 ctypes.byref(cs), int(max_tokens), _ptr(out), _stream(stream)),
            "kvarn_decode_attention_noalloc")
+    return out
+
+
+def decode_attention_multi(cfg: Config, q, cache: KVCache, max_tokens: int, out=None, workspace=None,
+                           softmax_scale: float = 0.0, stream=None):
+    """kvarn_decode_attention_multi: q [S, Q, Hq, D] (the last Q tokens of each sequence) -> out fp32, same shape."""
+    _need(q, "q", cfg.torch_dtype)
+    S, Q, Hq, D = q.shape
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32)
+    if workspace is None:
+        workspace = decode_workspace(cfg, Q * Hq, q.device)
+    c, cs = cfg.c(), cache.struct()
+    _check(lib().kvarn_decode_attention_multi(ctypes.byref(c), _ptr(q), int(Hq), int(Q), float(softmax_scale),
+                                              ctypes.byref(cs), int(max_tokens), _ptr(out), _ptr(workspace),
+                                              int(workspace.numel()), _stream(stream)),
+           "kvarn_decode_attention_multi")
     return out
 
 

@@ -201,6 +201,27 @@ KVARN_API int kvarn_decode_attention(const kvarn_config *cfg, const void *q, int
                            float *out, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Decode attention for several query tokens per sequence at once (draft
+ * tokens being verified, or a short chunk), the step next to single-token
+ * decode.  The queries are the last num_queries tokens already appended to
+ * the cache: for a sequence holding n tokens, query i (0-based) sits at
+ * position n - num_queries + i and attends positions 0 .. n - num_queries + i.
+ *   q    [num_seqs][num_queries][num_q_heads][D] in cfg->dtype, unrotated;
+ *   out  [num_seqs][num_queries][num_q_heads][D] fp32, unrotated.
+ * The num_queries x (num_q_heads / num_kv_heads) rows that share a kv head
+ * read its blocks once and fill the tensor-core tiles together; that count
+ * must be 1, 2, 4 or 8 (KVARN_EUNSUPPORTED otherwise).  Everything else --
+ * softmax_scale, max_tokens, status, empty sequences -- is as in
+ * kvarn_decode_attention; the workspace is
+ * kvarn_decode_workspace_bytes(cfg, num_queries * num_q_heads) bytes.  A
+ * query before position 0 (n < num_queries) gets zeros.
+ */
+KVARN_API int kvarn_decode_attention_multi(const kvarn_config *cfg, const void *q, int num_q_heads,
+                                           int num_queries, float softmax_scale, const kvarn_cache *cache,
+                                           int max_tokens, float *out, void *workspace, size_t workspace_bytes,
+                                           void *stream);
+
+/*
  * Quantisation error of stored blocks, per token, split into magnitude and
  * direction (article on KVarN, "The Problem": the errors that compound in
  * K are those of the token magnitudes, not of the directions; "How It

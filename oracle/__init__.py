@@ -227,6 +227,36 @@ def decode_from_cache(q, k_records, v_records, k_tail, v_tail, n_tokens: int, T:
     return attention(q, K, V, scale)
 
 
+def decode_multi_from_cache(q, k_records, v_records, k_tail, v_tail, n_tokens: int, T: int, hb: int,
+                            scale: float, group: int = 32, layouts=None) -> np.ndarray:
+    """Decode for the last Q tokens of one sequence at once: q (Q, Hq, D) -> out (Q, Hq, D).
+
+    The cache holds n_tokens tokens (blocks dequantised to the original basis, then the tail as stored); query i
+    sits at position n_tokens - Q + i and attends positions 0 .. n_tokens - Q + i (causal), by explicit softmax.
+    A query before position 0 gets zeros.
+    """
+    if layouts is None:
+        layouts = (K_ORDER, V_ORDER) if T == 128 else (NATURAL, NATURAL)
+    q = _f64(q)
+    Q, Hq, D = q.shape
+    Hkv = k_records.shape[0]
+    nblk, ntail = n_tokens // T, n_tokens % T
+    K = np.empty((Hkv, n_tokens, D))
+    V = np.empty((Hkv, n_tokens, D))
+    for h in range(Hkv):
+        for b in range(nblk):
+            K[h, b * T:(b + 1) * T] = dequantize_record(k_records[h, b], T, D, hb, False, layouts[0], group)
+            V[h, b * T:(b + 1) * T] = dequantize_record(v_records[h, b], T, D, hb, False, layouts[1], group)
+        K[h, nblk * T:] = np.asarray(k_tail[h, :ntail], dtype=np.float64)
+        V[h, nblk * T:] = np.asarray(v_tail[h, :ntail], dtype=np.float64)
+    out = np.zeros((Q, Hq, D))
+    for i in range(Q):
+        visible = n_tokens - Q + i + 1
+        if visible > 0:
+            out[i] = attention(q[i], K[:, :visible], V[:, :visible], scale)
+    return out
+
+
 # ------------------------------------------------------------ bulk, threads
 def quantize_many(x: np.ndarray, dtype: str, T: int, D: int, hb: int, sweeps: int = 4, group: int = 32,
                   nthreads: int = 1, layout: int = NATURAL):

@@ -403,3 +403,44 @@ def test_token_errors_match_oracle(D, hb, sweeps, dtype):
                 for b in range(2):
                     ref = oracle.record_token_errors(xs[s, h, b * 128:(b + 1) * 128], rs[s, h, b], 128, D, hb, lay)
                     np.testing.assert_allclose(es[s, h, b * 128:(b + 1) * 128], ref, rtol=1e-4, atol=2e-5)
+
+
+MQCASES = [
+    # name, S, H, Hq, Q, D, L, dtype, hb
+    ("gqa4_q2_tail41", 2, 2, 8, 2, 128, 3 * 128 + 41, torch.bfloat16, 128),
+    ("gqa4_q2_crosses_block", 2, 2, 8, 2, 128, 3 * 128, torch.bfloat16, 128),
+    ("gqa4_q2_block_edge", 1, 2, 8, 2, 128, 3 * 128 + 1, torch.bfloat16, 128),
+    ("gqa2_q4_crosses_block", 1, 2, 4, 4, 128, 2 * 128 + 2, torch.bfloat16, 128),
+    ("mha_q8_d96", 1, 4, 4, 8, 96, 2 * 128 + 3, torch.bfloat16, 32),
+    ("gqa8_q1", 1, 1, 8, 1, 128, 300, torch.bfloat16, 128),
+    ("q2_before_start", 2, 1, 4, 2, 64, 1, torch.float32, 64),
+]
+
+
+@pytest.mark.parametrize("case", MQCASES, ids=[c[0] for c in MQCASES])
+def test_multi_query_decode_matches_oracle(case):
+    name, S, H, Hq, Q, D, L, dtype, hb = case
+    k, v = _inputs(S, H, D, max(L, 1), dtype, 4, 0.5, (31, 32, 63, 64) if D == 96 else None, 300 + len(name))
+    q = synth.queries(301 + len(name), S * Q, Hq, D, dtype=dtype).reshape(S, Q, Hq, D)
+    cfg = _cfg(S, H, D, L // 128 + 1, dtype, hb)
+    cache, krec, vrec = _oracle_cache(cfg, k, v, L, hb)
+    out = kvarn.decode_attention_multi(cfg, q.to(DEV), cache, max_tokens=L).cpu().numpy()
+    assert int(cache.status.item()) == 0
+    kt, vt, qd = to_f64(cache.k_tail.cpu()), to_f64(cache.v_tail.cpu()), to_f64(q)
+    ref = np.stack([oracle.decode_multi_from_cache(qd[s], krec[s], vrec[s], kt[s], vt[s], L, 128, hb,
+                                                   1 / math.sqrt(D)) for s in range(S)])
+    err = float(np.max(np.abs(out - ref)))
+    print(name, "max abs err", err)
+    assert np.all(np.isfinite(out)) and err <= DECODE_ATOL
+    if Q == 1:  # one query is the single-token decode, bit for bit
+        single = kvarn.decode_attention(cfg, q[:, 0].contiguous().to(DEV), cache, max_tokens=L).cpu().numpy()
+        np.testing.assert_array_equal(out[:, 0], single)
+
+
+def test_multi_query_rows_beyond_eight_are_unsupported():
+    cfg = _cfg(1, 1, 128, 2, torch.bfloat16)
+    cache = kvarn.KVCache(cfg)
+    q = torch.zeros(1, 4, 4, 128, dtype=torch.bfloat16, device=DEV)  # 4 queries x GQA 4 = 16 rows
+    with pytest.raises(kvarn.KvarnError) as e:
+        kvarn.decode_attention_multi(cfg, q, cache, max_tokens=128, workspace=kvarn.decode_workspace(cfg, 8, DEV))
+    assert e.value.code == kvarn.KVARN_EUNSUPPORTED

@@ -402,3 +402,29 @@ def test_record_errors_vanish_on_the_grid_and_grow_without_normalisation():
         rec = oracle.pack_record(oracle.quantize_block(K, hb, sw))
         err[name] = oracle.record_token_errors(K, rec, T, D, hb).mean(axis=0)
     assert err["kvarn"][0] < err["rtn"][0]
+
+
+def test_multi_query_decode_is_causal_single_decodes():
+    """Q queries at once equal Q single-token decodes, each over the cache truncated after its own position; the
+    last query sees the whole cache."""
+    rng = np.random.default_rng(51)
+    T, D, Hkv, Hq, Q, n = 8, 64, 1, 2, 3, 17  # blocks 0-1 packed, one tail token; queries at positions 14, 15, 16
+    Kx = rng.standard_normal((Hkv, 24, D))
+    Vx = rng.standard_normal((Hkv, 24, D))
+    q = rng.standard_normal((Q, Hq, D))
+    krec = np.stack([[oracle.pack_record(oracle.quantize_block(Kx[0, b * T:(b + 1) * T], 64, 4)) for b in range(2)]])
+    vrec = np.stack([[oracle.pack_record(oracle.quantize_block(Vx[0, b * T:(b + 1) * T], 64, 4)) for b in range(2)]])
+    ktail = np.zeros((Hkv, T, D)); vtail = np.zeros((Hkv, T, D))
+    ktail[:, 0] = Kx[:, 16]; vtail[:, 0] = Vx[:, 16]
+    out = oracle.decode_multi_from_cache(q, krec, vrec, ktail, vtail, n, T, 64, 0.125)
+    np.testing.assert_allclose(out[Q - 1], oracle.decode_from_cache(q[Q - 1], krec, vrec, ktail, vtail, n, T, 64, 0.125),
+                               rtol=0, atol=1e-13)
+    Khat = np.concatenate([oracle.dequantize_record(krec[0, b], T, D, 64) for b in range(2)] + [Kx[0, 16:17]])
+    Vhat = np.concatenate([oracle.dequantize_record(vrec[0, b], T, D, 64) for b in range(2)] + [Vx[0, 16:17]])
+    for i in range(Q):
+        pos = n - Q + i
+        ref = oracle.attention(q[i], Khat[None, :pos + 1], Vhat[None, :pos + 1], 0.125)
+        np.testing.assert_allclose(out[i], ref, rtol=0, atol=1e-13)
+    # a query before position 0 gets zeros
+    z = oracle.decode_multi_from_cache(q, krec[:, :0], vrec[:, :0], ktail, vtail, 2, T, 64, 0.125)
+    assert np.all(z[0] == 0) and not np.all(z[2] == 0)
