@@ -169,11 +169,19 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             float2 s1 = f2(0.f, 0.f), s2 = f2(0.f, 0.f);
+            if (sw == 0) {  // c = 1: X / c is X
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float2 z = __fmul2_rn(X[r][k], u[k]);
-                s1 = __fadd2_rn(s1, z);
-                s2 = __ffma2_rn(z, z, s2);
+                for (int k = 0; k < 16; ++k) {
+                    s1 = __fadd2_rn(s1, X[r][k]);
+                    s2 = __ffma2_rn(X[r][k], X[r][k], s2);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const float2 z = __fmul2_rn(X[r][k], u[k]);
+                    s1 = __fadd2_rn(s1, z);
+                    s2 = __ffma2_rn(z, z, s2);
+                }
             }
             sm.part[sw & 1][j][l + 32 * r] = f2(s1.x + s1.y, s2.x + s2.y);
         }
