@@ -165,16 +165,16 @@ def run_kvarn(args, world, rank, local):
                 for _ in range(LAYERS)]
     probe_j = 64  # sub-step whose decode launches are bracketed with events
 
-    def step():
+    def step(qs_=qs, ks_=ks, vs_=vs, outs_=outs, probe=True):
         for c in caches:
             c.n_tokens.copy_(n_reset)
         for j in range(T_BLK):
             for layer, c in enumerate(caches):
-                kvarn.append_token(cfg, ks[j, layer], vs[j, layer], c)
-                if j == probe_j:
+                kvarn.append_token(cfg, ks_[j, layer], vs_[j, layer], c)
+                if probe and j == probe_j:
                     ev_pairs[layer][0].record()
-                kvarn.decode_attention(cfg, qs[j, layer], c, max_tokens=32768, out=outs[j, layer], workspace=ws)
-                if j == probe_j:
+                kvarn.decode_attention(cfg, qs_[j, layer], c, max_tokens=32768, out=outs_[j, layer], workspace=ws)
+                if probe and j == probe_j:
                     ev_pairs[layer][1].record()
 
     # ---- capture one step in a CUDA graph (9216 kernels), warm up
@@ -219,32 +219,63 @@ def run_kvarn(args, world, rank, local):
     peak, peak_kind = _peaks()
     achieved = dbytes / (dec_avg_ms / 1e3) / 1e9
 
-    # ---- end to end through the API: host (pinned) inputs in, outputs back, every step
+    # ---- end to end through the API: every step copies its inputs in from pinned host memory and its outputs
+    # back, as a serving loop does; with two buffer sets (and a graph for each) the copies of the neighbouring
+    # steps overlap this step's compute on their own streams
     h_q = torch.empty(qs.shape, dtype=qs.dtype, pin_memory=True).copy_(qs)
     h_k = torch.empty(ks.shape, dtype=ks.dtype, pin_memory=True).copy_(ks)
     h_v = torch.empty(vs.shape, dtype=vs.dtype, pin_memory=True).copy_(vs)
-    h_out = torch.empty(outs.shape, dtype=outs.dtype, pin_memory=True)
-    for _ in range(1):
-        qs.copy_(h_q, non_blocking=True); ks.copy_(h_k, non_blocking=True); vs.copy_(h_v, non_blocking=True)
-        graph.replay()
-        h_out.copy_(outs, non_blocking=True)
+    h_out = [torch.empty(outs.shape, dtype=outs.dtype, pin_memory=True) for _ in range(2)]
+    sets = [(qs, ks, vs, outs), tuple(torch.empty_like(t) for t in (qs, ks, vs, outs))]
+    graph_b = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_b, stream=stream):
+        step(*sets[1], probe=False)
+    graphs = [graph, graph_b]
+    h2d_s, d2h_s = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_run = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_steps(n, e_start=None, e_end=None):
+        if e_start is not None:
+            e_start.record(h2d_s)
+        for i in range(n):
+            b = i % 2
+            q_, k_, v_, o_ = sets[b]
+            with torch.cuda.stream(h2d_s):
+                if i >= 2:
+                    h2d_s.wait_event(ev_run[b])  # the step two back has read these inputs
+                q_.copy_(h_q, non_blocking=True); k_.copy_(h_k, non_blocking=True); v_.copy_(h_v, non_blocking=True)
+                ev_in[b].record(h2d_s)
+            with torch.cuda.stream(stream):
+                stream.wait_event(ev_in[b])
+                if i >= 2:
+                    stream.wait_event(ev_out[b])  # and its outputs have been read back
+                graphs[b].replay()
+                ev_run[b].record(stream)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(ev_run[b])
+                h_out[b].copy_(o_, non_blocking=True)
+                ev_out[b].record(d2h_s)
+        if e_end is not None:
+            d2h_s.wait_stream(stream)
+            e_end.record(d2h_s)
+
+    e2e_steps(2)
     torch.cuda.synchronize()
     _barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        qs.copy_(h_q, non_blocking=True); ks.copy_(h_k, non_blocking=True); vs.copy_(h_v, non_blocking=True)
-        graph.replay()
-        h_out.copy_(outs, non_blocking=True)
-    e1.record()
+    e2e_steps(args.steps, e0, e1)
     torch.cuda.synchronize()
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1), world)
     e2e_value = dp.aggregate_rate(S * T_BLK * args.steps, e2e_ms / 1e3, world)
+    if not torch.equal(h_out[(args.steps - 1) % 2], sets[(args.steps - 1) % 2][3].cpu()):
+        raise RuntimeError("end-to-end outputs read back do not match the device outputs")
     h2d = (qs.numel() + ks.numel() + vs.numel()) * 2
     d2h = outs.numel() * 4
-    del graph
+    del graph, graph_b, graphs
     caches.clear()
-    del qs, ks, vs, outs, ws, h_q, h_k, h_v, h_out
+    del qs, ks, vs, outs, ws, h_q, h_k, h_v, h_out, sets
     torch.cuda.empty_cache()
 
     # ---- bulk quantise GB/s (Llama-3-8B-shaped prefill)

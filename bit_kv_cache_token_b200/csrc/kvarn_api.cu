@@ -12,7 +12,7 @@ namespace {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Shape / method checks shared by every call.  EUNSUPPORTED for well-formed
-// parameters this build has no kernel for, EINVAL for malformed ones.
+// parameters the library has no kernel for, EINVAL for malformed ones.
 int check_config(const kvarn_config *c)
 {
     if (!c) return KVARN_EINVAL;
