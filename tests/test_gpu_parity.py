@@ -444,3 +444,23 @@ def test_multi_query_rows_beyond_eight_are_unsupported():
     with pytest.raises(kvarn.KvarnError) as e:
         kvarn.decode_attention_multi(cfg, q, cache, max_tokens=128, workspace=kvarn.decode_workspace(cfg, 8, DEV))
     assert e.value.code == kvarn.KVARN_EUNSUPPORTED
+
+
+def test_decode_many_short_sequences():
+    """1024 (sequence, kv head) units of 300 tokens: more items than warps, so warp ranges cross units and
+    partials merge warp by warp.  Sampled units against the oracle decoding the records the GPU wrote."""
+    S, H, Hq, D, L = 128, 8, 32, 128, 300
+    k, v = synth.layer_kv(700, 0, S, H, L, D, n_outliers=4, device=DEV)
+    q = synth.queries(701, S, Hq, D, device=DEV)
+    cfg = _cfg(S, H, D, 3, torch.bfloat16)
+    cache = kvarn.KVCache(cfg)
+    kvarn.quantize_blocks(cfg, k, v, cache)
+    out = kvarn.decode_attention(cfg, q, cache, max_tokens=L).cpu().numpy()
+    torch.cuda.synchronize()
+    assert int(cache.status.item()) == 0 and np.all(np.isfinite(out))
+    rng = np.random.default_rng(702)
+    kr, vr = cache.k_records.cpu().numpy(), cache.v_records.cpu().numpy()
+    kt, vt, qd = to_f64(cache.k_tail.cpu()), to_f64(cache.v_tail.cpu()), to_f64(q.cpu())
+    for s in sorted({int(x) for x in rng.integers(0, S, 6)} | {0, S - 1}):
+        ref = oracle.decode_from_cache(qd[s], kr[s], vr[s], kt[s], vt[s], L, 128, 128, 1 / math.sqrt(D))
+        assert np.max(np.abs(out[s] - ref)) <= DECODE_ATOL
