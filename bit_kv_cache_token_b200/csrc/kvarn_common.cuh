@@ -65,11 +65,14 @@ struct In;
 
 template <>
 struct In<float> {
-    // load 8 consecutive elements (32 bytes, 16-byte aligned) as fp32
+    // load 8 consecutive elements (32 bytes, 16-byte aligned) as fp32; COHERENT
+    // reads through L2 (data this kernel may have written), else the read-only path
+    template <bool COHERENT = false>
     static __device__ __forceinline__ void load8(const float *p, float (&o)[8])
     {
-        const float4 a = __ldg(reinterpret_cast<const float4 *>(p));
-        const float4 b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+        const float4 *q = reinterpret_cast<const float4 *>(p);
+        const float4 a = COHERENT ? __ldcg(q) : __ldg(q);
+        const float4 b = COHERENT ? __ldcg(q + 1) : __ldg(q + 1);
         o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
         o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
     }
@@ -85,9 +88,11 @@ struct In<float> {
 
 template <>
 struct In<__nv_bfloat16> {
+    template <bool COHERENT = false>
     static __device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&o)[8])
     {
-        const uint4 a = __ldg(reinterpret_cast<const uint4 *>(p));
+        const uint4 *q = reinterpret_cast<const uint4 *>(p);
+        const uint4 a = COHERENT ? __ldcg(q) : __ldg(q);
         const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {

@@ -66,7 +66,7 @@ append_kernel(AppendArgs a)
         if (fills) {
             __syncthreads();  // the new row is visible to the whole CTA
             float2 X[4][16];
-            load_block<D>(tail, X);
+            load_block<D, Tin, true>(tail, X);  // row pos was just written by this CTA
             unsigned char *rec = static_cast<unsigned char *>(tensor ? a.v_records : a.k_records) +
                                  ((size_t)sh * a.max_blocks + blk) * Record<D>::kBytes;
             if (tensor) quantize_block<D, HB, 1>(X, sm, a.sweeps, rec, nullptr, a.status);

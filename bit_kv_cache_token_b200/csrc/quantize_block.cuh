@@ -77,7 +77,9 @@ __device__ __forceinline__ void fwht32_regs(float2 (&x)[16])
 
 // Load a block of 128 rows x D channels (row stride D elements) into the
 // thread layout described above.  `rows` may be a device or tail buffer.
-template <int D, typename Tin>
+// COHERENT: the rows may have been written by this kernel (the append path's
+// tail), so they are read through L2 rather than the read-only path.
+template <int D, typename Tin, bool COHERENT = false>
 __device__ __forceinline__ void load_block(const Tin *rows, float2 (&X)[4][16])
 {
     const int j = threadIdx.x >> 5, l = threadIdx.x & 31;
@@ -87,7 +89,7 @@ __device__ __forceinline__ void load_block(const Tin *rows, float2 (&X)[4][16])
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             float v[8];
-            In<Tin>::load8(p + 8 * q, v);
+            In<Tin>::template load8<COHERENT>(p + 8 * q, v);
 #pragma unroll
             for (int e = 0; e < 4; ++e) X[r][4 * q + e] = f2(v[2 * e], v[2 * e + 1]);
         }
