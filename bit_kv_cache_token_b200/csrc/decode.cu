@@ -25,19 +25,23 @@
 // copy overlaps half a block of this warp's work and the whole work of the
 // SM's other warps.  Both contractions run on tensor cores (mma.sync
 // m16n8k16, fp16 in, fp32 accumulate):
-//   scores: A = q' (rows: query heads; hi/lo fp16 split in rows 0-7 / 8-15),
-//           B = K codes (k = channels, n = 8 tokens);
-//   P V:    A = p r s (rows: heads, hi/lo), B = V codes (k = tokens, n = 8 channels).
+//   scores: A = K codes (16 tokens x 16 channels), B = q' (16 channels x 8
+//           columns: a column per head and hi/lo fp16 part), one accumulator
+//           per 32-channel group, scaled by s r in the epilogue;
+//   P V:    A = p r s (rows: heads and hi/lo parts), B = V codes (k = 16
+//           tokens, n = 8 channels); the probabilities move from the score
+//           layout to these rows by shuffles.
 // A 2-bit code becomes an exact fp16 operand with a shift and an AND: the
 // record stores every code in a 32-bit word at bit 16*half + 2*pos (see
 // kvarn.h), and masking a shifted copy of the word puts both codes of a pair
 // on bits 8-9 or 6-7 of their halves, i.e. fp16 subnormals c * 2^-16 or
 // c * 2^-18.  The factor 4 between the two is folded into the other operand
 // (it depends only on the contracted index), the remaining 2^-16 into the
-// scales.  When the GQA group has fewer than 8 heads, the spare rows
-// carry copies of the heads working on other channel groups, so every lane
-// does useful work.  The tail item is attended on CUDA cores with
-// load-parallel loops.
+// scales.  When the GQA group has fewer than 8 heads, the spare P V rows
+// carry copies of the heads working on other channel groups.  The tail item
+// is attended on CUDA cores with load-parallel loops.  Several query tokens
+// per sequence (MQ instantiations) are more rows on the same kv head, with a
+// causal limit applied in the last block and the tail.
 //
 // Merging.  Every (warp, unit) segment writes one partial (m, l, o_rot per
 // head); the tail item writes the unit's tail partial.  A per-unit ticket
@@ -349,7 +353,6 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
     using R = Record<D>;
     constexpr int NG = D / kGroup;          // channel groups
     constexpr int NKT = D / 16;             // k-tiles of the score MMA
-    constexpr int NNT = D / 8;              // n-tiles of the P V MMA
     constexpr int C = 8 / GRP;              // head copies in the 8 rows of the P V MMA
     constexpr int SETS = (NG + C - 1) / C;  // groups handled per copy
     constexpr int KW = D / 32;              // K code words per (16-token unit, lane)
