@@ -523,7 +523,7 @@ def main():
             runs.append(oracle_sample())
         val = statistics.median(r["value"] for r in runs)
         line = {"metric": METRIC, "value": val, "unit": UNIT, "n_gpus": 0, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": S * T_BLK / val * 1e3,  # extrapolated from the sample "higher_is_better": True, "scaling": "weak",
+                "warmup": args.warmup, "ms_per_step": S * T_BLK / val * 1e3, "higher_is_better": True, "scaling": "weak",  # ms_per_step: extrapolated from the sample
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
                 "config": {"workload": WORKLOAD, "global_batch": S, "seq_len": 32768},
                 "cpu_baseline": {k: runs[-1][k] for k in ("value", "unit", "cores", "kind", "sample")},
