@@ -541,10 +541,12 @@ def main():
         line = {
             "metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": r["ms_step"], "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16 in, 2-bit cache, fp32 math", "data": "synthetic",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "global_batch": S * world, "seq_len": 32768, "layers": LAYERS,
                        "q_heads": HQ, "kv_heads": HKV, "head_dim": D, "tokens_per_step": S * T_BLK * world,
                        "parallelism": f"dp{world} (independent batches, no collective)",
+                       "numerics": "bf16 inputs, 2-bit records with binary16 scales, fp32 arithmetic (tensor-core "
+                                   "operands as fp16 hi/lo pairs, fp32 accumulation)",
                        "l2": "inputs larger than L2: each decode launch streams ~219 MB of cache, 7.9 GB per token"},
             "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": r["achieved"], "peak": r["peak"],
                          "unit": "GB/s", "frac": r["achieved"] / r["peak"], "traffic": DECODE_TRAFFIC_BYTES,
