@@ -50,11 +50,12 @@ def _bf16_bits(t: torch.Tensor) -> np.ndarray:
     return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
 
 
-def _decode_layer(S, H, Hq, D, hb, ctx, appended, seed, n_out, max_blocks, max_tokens, fixed=None, samples=4):
+def _decode_layer(S, H, Hq, D, hb, ctx, appended, seed, n_out, max_blocks, max_tokens, fixed=None, samples=4,
+                  layer=0):
     """Prefill ctx tokens in bulk, append the rest one at a time, decode; compare sampled units with the oracle."""
     total = ctx + appended
     cfg = kvarn.Config(S, H, D, max_blocks=max_blocks, hadamard=hb)
-    k, v = synth.layer_kv(seed, 0, S, H, total, D, n_outliers=n_out, outlier_channels=fixed, device="cuda")
+    k, v = synth.layer_kv(seed, layer, S, H, total, D, n_outliers=n_out, outlier_channels=fixed, device="cuda")
     cache = kvarn.KVCache(cfg)
     kvarn.quantize_blocks(cfg, k[:, :, :ctx].contiguous(), v[:, :, :ctx].contiguous(), cache)
     for t in range(ctx, total):
@@ -97,6 +98,16 @@ def _decode_layer(S, H, Hq, D, hb, ctx, appended, seed, n_out, max_blocks, max_t
 def test_qwen_decode_layer_32k_sampled():
     # context 32705 as in the benchmark's probe sub-step; block 254 quantised by the append path, 65 tail tokens
     print("max abs err", _decode_layer(8, 8, 32, 128, 128, 32512, 193, 2, 4, max_blocks=256, max_tokens=32768))
+
+
+@pytest.mark.parametrize("total,layer", [(1024, 0), (1151, 35), (4153, 0), (32768, 35)])
+def test_qwen_decode_at_checkpoint_contexts(total, layer):
+    """The Qwen3-4B-shaped batch (8 sequences, 8 kv / 32 q heads) at the checkpoint contexts, first and last layer:
+    bulk prefill of the whole blocks but the last, the rest appended token by token."""
+    ctx = (total // 128 - 1) * 128 if total >= 256 else 0
+    err = _decode_layer(8, 8, 32, 128, 128, ctx, total - ctx, 40 + layer, 4, max_blocks=256, max_tokens=total,
+                        samples=2, layer=layer)
+    print(total, layer, "max abs err", err)
 
 
 def test_phi_mha_decode_layer_16k_sampled():
