@@ -1,8 +1,8 @@
 """Parity at the full benchmark sizes, on sampled outputs the oracle computes one by one.
 
 * Bulk quantisation of the Llama-3-8B-shaped prefill (batch 32 x 32 layers x 8 kv heads x 8192 tokens,
-  head_dim 128, bf16, K token sigma 0.7), in the single launch the benchmark times: sampled blocks against the
-  oracle (codes outside the 1e-5 rounding window and binary16 scales away from a rounding midpoint, exact).
+  head_dim 128, bf16, K token sigma 0.7), in the single launch the benchmark times: 256 seeded random blocks and the
+  first and last, K and V, against the oracle (codes outside the 1e-5 rounding window and binary16 scales away from a rounding midpoint, exact).
 * One Qwen3-4B-shaped decode layer at a 32K context (batch 8, 32 q / 8 kv heads), built as the benchmark builds
   it: bulk prefill, then appended tokens (one of them quantises block 254), decode at context 32705 with the
   benchmark's max_tokens.  Sampled (sequence, kv head) pairs get oracle-packed records on the same
@@ -37,7 +37,7 @@ def test_llama_bulk_quantise_full_size_sampled():
     torch.cuda.synchronize()
     assert int(cache.status.item()) == 0
     rng = np.random.default_rng(0)
-    picks = [(int(rng.integers(nseq)), int(rng.integers(H)), int(rng.integers(T // 128))) for _ in range(48)]
+    picks = [(int(rng.integers(nseq)), int(rng.integers(H)), int(rng.integers(T // 128))) for _ in range(256)]
     picks += [(0, 0, 0), (nseq - 1, H - 1, T // 128 - 1)]
     for s, h, b in picks:
         for tensor, x, recs, lay in ((0, k, cache.k_records, oracle.K_ORDER), (1, v, cache.v_records, oracle.V_ORDER)):
