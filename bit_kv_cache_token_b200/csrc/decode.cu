@@ -58,7 +58,9 @@ namespace kvarn {
 
 constexpr float kTwo16 = 65536.f;           // 2^16
 constexpr float kTwoM16 = 1.f / 65536.f;    // 2^-16
-constexpr long long kWaitLimit = 1LL << 26; // bounded mbarrier polling
+// Longest wait for a staged record, in ns of the global timer (a record
+// normally lands within microseconds).
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 template <int D, int GRP>
 struct alignas(128) DecWarpSmem {
@@ -201,19 +203,34 @@ __device__ __forceinline__ void issue_record(unsigned long long *bar, unsigned c
                  : "memory");
 }
 
-// Bounded wait for phase `parity` of an mbarrier; false if the limit ran out.
-__device__ __forceinline__ bool mbar_wait(unsigned long long *bar, uint32_t parity)
+__device__ __forceinline__ bool mbar_try(unsigned long long *bar, uint32_t parity)
 {
-    for (long long i = 0; i < kWaitLimit; ++i) {
-        uint32_t done;
-        asm volatile(
-            "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-            : "=r"(done)
-            : "r"(smem_u32(bar)), "r"(parity)
-            : "memory");
-        if (done) return true;
+    uint32_t done;
+    asm volatile("{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+                 : "=r"(done)
+                 : "r"(smem_u32(bar)), "r"(parity)
+                 : "memory");
+    return done != 0u;
+}
+
+__device__ __forceinline__ unsigned long long global_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait for phase `parity` of an mbarrier: false once limit_ns of the
+// global timer have passed without it.  The timer is read only when the
+// first try does not succeed.
+__device__ __forceinline__ bool mbar_wait(unsigned long long *bar, uint32_t parity, unsigned long long limit_ns)
+{
+    if (mbar_try(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    for (unsigned it = 1;; ++it) {
+        if (mbar_try(bar, parity)) return true;
+        if ((it & 63u) == 0u && global_ns() - t0 > limit_ns) return false;
     }
-    return false;
 }
 
 // Normalised Walsh-Hadamard transform (block hb, 0 = none) of nvec rows of
@@ -348,7 +365,7 @@ template <int D, int GRP, typename Tin, bool MQ>
 __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, const unsigned char *vbase, int b0,
                            int b1, uint32_t &kph, uint32_t &vph, float (&m_run)[(GRP + 3) / 4],
                            float (&l_run)[(GRP + 3) / 4], float2 (&orun)[dec_sets<D, GRP>()][kGroup / 8],
-                           int blim0, int hpk)
+                           int blim0, int hpk, unsigned long long wait_ns, bool withhold_k)
 {
     using R = Record<D>;
     constexpr int NG = D / kGroup;          // channel groups
@@ -366,13 +383,17 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
 
     if (b0 >= b1) return true;
     if (lane == 0) {
-        issue_record(&sm.mbar[0], sm.rec[0], kbase + (size_t)b0 * R::kBytes, R::kBytes);
+        if (!withhold_k)  // self-test of the bounded wait: the first K record is never requested
+            issue_record(&sm.mbar[0], sm.rec[0], kbase + (size_t)b0 * R::kBytes, R::kBytes);
         issue_record(&sm.mbar[1], sm.rec[1], vbase + (size_t)b0 * R::kBytes, R::kBytes);
     }
     for (int b = b0; b < b1; ++b) {
-        if (!mbar_wait(&sm.mbar[0], kph)) {
-            // in flight: K and V of block b
-            if (lane == 0) { mbar_wait(&sm.mbar[0], kph); mbar_wait(&sm.mbar[1], vph); }
+        if (!mbar_wait(&sm.mbar[0], kph, wait_ns)) {
+            // in flight: K (unless withheld) and V of block b
+            if (lane == 0) {
+                if (!withhold_k) mbar_wait(&sm.mbar[0], kph, wait_ns);
+                mbar_wait(&sm.mbar[1], vph, wait_ns);
+            }
             __syncwarp();
             return false;
         }
@@ -559,11 +580,11 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
         __syncwarp();  // every lane is done with the K record and the K scales
         if (lane == 0 && b + 1 < b1)
             issue_record(&sm.mbar[0], sm.rec[0], kbase + (size_t)(b + 1) * R::kBytes, R::kBytes);
-        if (!mbar_wait(&sm.mbar[1], vph)) {
+        if (!mbar_wait(&sm.mbar[1], vph, wait_ns)) {
             // in flight: V of block b and K of block b + 1
             if (lane == 0) {
-                mbar_wait(&sm.mbar[1], vph);
-                if (b + 1 < b1) mbar_wait(&sm.mbar[0], kph);
+                mbar_wait(&sm.mbar[1], vph, wait_ns);
+                if (b + 1 < b1) mbar_wait(&sm.mbar[0], kph, wait_ns);
             }
             __syncwarp();
             return false;
@@ -1099,7 +1120,8 @@ decode_kernel(DecodeArgs a, int hb)
             const unsigned char *vbase =
                 static_cast<const unsigned char *>(a.v_records) + (size_t)unit * a.max_blocks * R::kBytes;
             if (!run_blocks<D, GRP, Tin, MQ>(sm, kbase, vbase, b0, b1r, kph, vph, m_run, l_run, orun, n - a.num_queries,
-                                         a.heads_per_kv)) {
+                                             a.heads_per_kv, a.wait_ns ? a.wait_ns : kWaitLimitNs,
+                                             a.withhold_first_k != 0)) {
                 dead = true;
                 if (lane == 0) status_or(a.status, KVARN_STATUS_TIMEOUT);
 #pragma unroll

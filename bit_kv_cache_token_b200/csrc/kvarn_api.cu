@@ -146,7 +146,7 @@ int kvarn_append_token(const kvarn_config *cfg, const void *k, const void *v, co
 
 static int decode_impl(const kvarn_config *cfg, const void *q, int num_q_heads, int num_queries,
                        float softmax_scale, const kvarn_cache *cache, int max_tokens, float *out, void *workspace,
-                       size_t workspace_bytes, void *stream)
+                       size_t workspace_bytes, void *stream, unsigned long long wait_ns = 0, int withhold = 0)
 {
     int rc = check_config(cfg);
     if (rc) return rc;
@@ -183,6 +183,7 @@ static int decode_impl(const kvarn_config *cfg, const void *q, int num_q_heads, 
     a.num_kv_heads = cfg->num_kv_heads; a.grp = rows; a.max_blocks = cfg->max_blocks;
     a.max_tokens = max_tokens; a.num_units = units;
     a.num_queries = num_queries; a.heads_per_kv = hpk;
+    a.wait_ns = wait_ns; a.withhold_first_k = withhold;
     return cuda_status(run_decode(*cfg, a, ctas, static_cast<cudaStream_t>(stream)));
 }
 
@@ -192,6 +193,14 @@ int kvarn_decode_attention(const kvarn_config *cfg, const void *q, int num_q_hea
 {
     return decode_impl(cfg, q, num_q_heads, 1, softmax_scale, cache, max_tokens, out, workspace, workspace_bytes,
                        stream);
+}
+
+int kvarn_decode_selftest_timeout(const kvarn_config *cfg, const void *q, int num_q_heads, const kvarn_cache *cache,
+                                  int max_tokens, float *out, void *workspace, size_t workspace_bytes, void *stream)
+{
+    // every warp's first K record is withheld and its wait ends after 1 ms
+    return decode_impl(cfg, q, num_q_heads, 1, 0.f, cache, max_tokens, out, workspace, workspace_bytes, stream,
+                       1000000ull, 1);
 }
 
 int kvarn_decode_attention_multi(const kvarn_config *cfg, const void *q, int num_q_heads, int num_queries,

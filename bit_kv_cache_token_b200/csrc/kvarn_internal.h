@@ -53,6 +53,10 @@ struct DecodeArgs {
     // q and out are [S][num_queries][Hq][D]; query i of a sequence with n
     // tokens sits at position n - num_queries + i and sees positions <= it.
     int num_queries, heads_per_kv;
+    // Bounded waits: limit per staged-record wait in ns (0 = the default) and,
+    // for the self-test only, a flag that withholds each segment's first K copy.
+    unsigned long long wait_ns;
+    int withhold_first_k;
 };
 
 struct ErrorArgs {

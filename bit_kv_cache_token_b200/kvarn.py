@@ -33,6 +33,7 @@ EXPORTED = (
     "kvarn_record_bytes", "kvarn_cache_bytes", "kvarn_decode_workspace_bytes", "kvarn_quantize_blocks",
     "kvarn_append_token", "kvarn_decode_attention", "kvarn_dequantize", "kvarn_strerror",
     "kvarn_decode_attention_noalloc", "kvarn_token_errors", "kvarn_decode_attention_multi",
+    "kvarn_decode_selftest_timeout",
 )
 
 
@@ -78,6 +79,7 @@ def lib() -> ctypes.CDLL:
         L.kvarn_decode_attention_noalloc.argtypes = [P(kvarn_config), V, I, F, P(kvarn_cache), I, V, V]
         L.kvarn_token_errors.argtypes = [P(kvarn_config), V, V, I, I, P(kvarn_cache), V, V, V]
         L.kvarn_decode_attention_multi.argtypes = [P(kvarn_config), V, I, I, F, P(kvarn_cache), I, V, V, S, V]
+        L.kvarn_decode_selftest_timeout.argtypes = [P(kvarn_config), V, I, P(kvarn_cache), I, V, V, S, V]
         L.kvarn_strerror.argtypes = [I]
         L.kvarn_strerror.restype = ctypes.c_char_p
         for name in ("kvarn_quantize_blocks", "kvarn_append_token", "kvarn_decode_attention", "kvarn_dequantize",
@@ -266,6 +268,20 @@ def decode_attention_multi(cfg: Config, q, cache: KVCache, max_tokens: int, out=
                                               ctypes.byref(cs), int(max_tokens), _ptr(out), _ptr(workspace),
                                               int(workspace.numel()), _stream(stream)),
            "kvarn_decode_attention_multi")
+    return out
+
+
+def decode_selftest_timeout(cfg: Config, q, cache: KVCache, max_tokens: int, stream=None):
+    """kvarn_decode_selftest_timeout: decode with every first K copy withheld and 1 ms waits; returns the output
+    (not meaningful) -- the caller checks KVARN_STATUS_TIMEOUT in cache.status."""
+    _need(q, "q", cfg.torch_dtype)
+    Hq = q.shape[1]
+    out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    workspace = decode_workspace(cfg, Hq, q.device)
+    c, cs = cfg.c(), cache.struct()
+    _check(lib().kvarn_decode_selftest_timeout(ctypes.byref(c), _ptr(q), int(Hq), ctypes.byref(cs), int(max_tokens),
+                                               _ptr(out), _ptr(workspace), int(workspace.numel()), _stream(stream)),
+           "kvarn_decode_selftest_timeout")
     return out
 
 

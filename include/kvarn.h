@@ -59,8 +59,8 @@ extern "C" {
 #define KVARN_STATUS_CAPACITY  1  /* append needed block >= max_blocks     */
 #define KVARN_STATUS_NONFINITE 2  /* a scale rounded to inf/nan in binary16 */
 #define KVARN_STATUS_LENGTH    4  /* n_tokens[s] > max_tokens at decode     */
-#define KVARN_STATUS_TIMEOUT   8  /* a staged copy did not arrive in time;  */
-                                  /* the affected partial result is dropped */
+#define KVARN_STATUS_TIMEOUT   8  /* a staged copy did not arrive within  */
+                                  /* 2 s; the affected partial is dropped   */
 
 typedef enum { KVARN_F32 = 0, KVARN_BF16 = 1 } kvarn_dtype;
 
@@ -220,6 +220,20 @@ KVARN_API int kvarn_decode_attention_multi(const kvarn_config *cfg, const void *
                                            int num_queries, float softmax_scale, const kvarn_cache *cache,
                                            int max_tokens, float *out, void *workspace, size_t workspace_bytes,
                                            void *stream);
+
+/*
+ * Self-test of the decode kernel's bounded waits (an engineering check; the
+ * method has no counterpart).  Runs kvarn_decode_attention with every warp's
+ * first K record copy withheld and each staged-record wait limited to 1 ms
+ * of the global timer (the normal limit is 2 s).  The launch must end -- not
+ * hang -- with KVARN_STATUS_TIMEOUT OR-ed into *cache->status; the outputs
+ * are not meaningful.  Afterwards the context and the cache stay usable: a
+ * normal decode on the same cache gives its usual result.  Arguments and
+ * errors as kvarn_decode_attention (softmax scale 1/sqrt(D)).
+ */
+KVARN_API int kvarn_decode_selftest_timeout(const kvarn_config *cfg, const void *q, int num_q_heads,
+                                            const kvarn_cache *cache, int max_tokens, float *out, void *workspace,
+                                            size_t workspace_bytes, void *stream);
 
 /*
  * Quantisation error of stored blocks, per token, split into magnitude and

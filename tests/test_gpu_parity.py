@@ -464,3 +464,25 @@ def test_decode_many_short_sequences():
     for s in sorted({int(x) for x in rng.integers(0, S, 6)} | {0, S - 1}):
         ref = oracle.decode_from_cache(qd[s], kr[s], vr[s], kt[s], vt[s], L, 128, 128, 1 / math.sqrt(D))
         assert np.max(np.abs(out[s] - ref)) <= DECODE_ATOL
+
+
+def test_bounded_wait_ends_with_timeout_status_and_leaves_context_usable():
+    """A staged record that never arrives (the self-test withholds each warp's first K copy, 1 ms limit) ends the
+    launch with KVARN_STATUS_TIMEOUT instead of a hang; a normal decode afterwards gives its usual result."""
+    S, H, Hq, D, L = 2, 2, 8, 128, 1000
+    k, v = _inputs(S, H, D, L, torch.bfloat16, 4, 0.5, None, 800)
+    q = synth.queries(801, S, Hq, D).to(DEV)
+    cfg = _cfg(S, H, D, L // 128 + 1, torch.bfloat16)
+    cache = kvarn.KVCache(cfg)
+    kvarn.quantize_blocks(cfg, k.to(DEV), v.to(DEV), cache)
+    ref = kvarn.decode_attention(cfg, q, cache, max_tokens=L).cpu()
+    torch.cuda.synchronize()
+    assert int(cache.status.item()) == 0
+    kvarn.decode_selftest_timeout(cfg, q, cache, max_tokens=L)
+    torch.cuda.synchronize()
+    assert int(cache.status.item()) & kvarn.KVARN_STATUS_TIMEOUT
+    cache.status.zero_()
+    again = kvarn.decode_attention(cfg, q, cache, max_tokens=L).cpu()
+    torch.cuda.synchronize()
+    assert int(cache.status.item()) == 0
+    assert torch.equal(again, ref)
