@@ -41,7 +41,7 @@ QB_WORKLOAD = "Llama-3-8B-shaped bulk prefill quantise: 32 batch x 32 layers x 8
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one decode launch at context 32705 for this
 # batch, from one ncu capture of `bench.py --profile decode` with the current decode kernel; reset it to None
 # whenever the decode kernel changes until it is captured again.
-DECODE_TRAFFIC_BYTES = None  # decode kernel changed since the last capture
+DECODE_TRAFFIC_BYTES = 219929856 + 4410112
 
 
 def _peaks():
