@@ -1,4 +1,5 @@
 // kvarn_api.cu -- the extern "C" boundary: validation, sizes, launches.
+#include <limits.h>
 #include <math.h>
 #include <stdint.h>
 
@@ -60,6 +61,12 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? KVARN_OK : KVARN_ECUD
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// One CTA per (sequence, kv head, block): the grid's x extent must fit an int.
+bool grid_fits(const kvarn_config *c, long long blocks_per_unit)
+{
+    return (long long)c->num_seqs * c->num_kv_heads * blocks_per_unit <= INT_MAX;
+}
+
 size_t ticket_bytes(const kvarn_config *c)
 {
     return align_up((size_t)c->num_seqs * c->num_kv_heads * sizeof(uint32_t), 256);
@@ -113,6 +120,7 @@ int kvarn_quantize_blocks(const kvarn_config *cfg, const void *k, const void *v,
     if (num_tokens < 0 || first_block < 0) return KVARN_EINVAL;
     if (num_tokens > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return KVARN_EINVAL;
     if ((long long)first_block + num_tokens / cfg->block_tokens > cfg->max_blocks) return KVARN_EINVAL;
+    if (!grid_fits(cfg, num_tokens / cfg->block_tokens + 1)) return KVARN_EINVAL;
     if ((debug_k && !aligned16(debug_k)) || (debug_v && !aligned16(debug_v))) return KVARN_EINVAL;
     QuantArgs a;
     a.k = k; a.v = v;
@@ -219,7 +227,7 @@ int kvarn_token_errors(const kvarn_config *cfg, const void *k, const void *v, in
     if ((rc = check_cache(cache, false))) return rc;
     if (num_tokens < 0 || num_tokens % cfg->block_tokens || first_block < 0) return KVARN_EINVAL;
     const int nb = num_tokens / cfg->block_tokens;
-    if ((long long)first_block + nb > cfg->max_blocks) return KVARN_EINVAL;
+    if ((long long)first_block + nb > cfg->max_blocks || !grid_fits(cfg, nb)) return KVARN_EINVAL;
     if (nb == 0) return KVARN_OK;
     if (!k || !v || !err_k || !err_v || !aligned16(k) || !aligned16(v) || !aligned16(err_k) || !aligned16(err_v))
         return KVARN_EINVAL;
@@ -239,6 +247,7 @@ int kvarn_dequantize(const kvarn_config *cfg, const kvarn_cache *cache, int firs
     if (!cache || !cache->k_records || !cache->v_records) return KVARN_EINVAL;
     if (first_block < 0 || num_blocks < 0 || (long long)first_block + num_blocks > cfg->max_blocks)
         return KVARN_EINVAL;
+    if (!grid_fits(cfg, num_blocks)) return KVARN_EINVAL;
     if ((k_out && !aligned16(k_out)) || (v_out && !aligned16(v_out))) return KVARN_EINVAL;
     DequantArgs a;
     a.k_records = cache->k_records; a.v_records = cache->v_records;

@@ -161,7 +161,8 @@ KVARN_API size_t kvarn_decode_workspace_bytes(const kvarn_config *cfg, int num_q
  * record slots first_block, first_block+1, ...; the last num_tokens % T
  * tokens are copied, unrotated, into the tail; n_tokens[s] is set to
  * first_block*T + num_tokens.  Needs first_block + floor(num_tokens/T) <=
- * max_blocks (KVARN_EINVAL otherwise).
+ * max_blocks, and num_seqs*num_kv_heads*(floor(num_tokens/T) + 1) <= INT_MAX
+ * (one CTA per block and tail; KVARN_EINVAL otherwise).
  * debug_k / debug_v: NULL, or fp32 buffers of
  *   num_seqs*num_kv_heads*(num_tokens/T) * (T + D + 2*T*(D/group)) floats
  *   receiving, per block, the unrounded r[T], c[D], s[T][D/group],
@@ -250,7 +251,8 @@ KVARN_API int kvarn_decode_selftest_timeout(const kvarn_config *cfg, const void 
  * quantiser rotates it and x^ = r c (s code + m) from the stored binary16
  * scales.  Useful with cfg->hadamard = 0 or cfg->sweeps = 0 to measure what
  * each stage removes.  Errors: KVARN_EINVAL for a ragged num_tokens, a block
- * range beyond max_blocks, or a NULL / unaligned pointer.
+ * range beyond max_blocks, num_seqs*num_kv_heads*num_tokens/T above INT_MAX,
+ * or a NULL / unaligned pointer.
  */
 KVARN_API int kvarn_token_errors(const kvarn_config *cfg, const void *k, const void *v, int num_tokens,
                                  int first_block, const kvarn_cache *cache, float *err_k, float *err_v,
@@ -260,7 +262,9 @@ KVARN_API int kvarn_token_errors(const kvarn_config *cfg, const void *k, const v
  * Dequantise records first_block .. first_block+num_blocks-1 of every
  * (sequence, kv head) into fp32 k_out / v_out
  * [num_seqs][num_kv_heads][num_blocks*T][D]; rotated != 0 keeps the rotated
- * basis, rotated == 0 rotates back.  Either output may be NULL.
+ * basis, rotated == 0 rotates back.  Either output may be NULL.  Errors:
+ * KVARN_EINVAL for a block range outside 0 .. max_blocks, or
+ * num_seqs*num_kv_heads*num_blocks above INT_MAX.
  */
 KVARN_API int kvarn_dequantize(const kvarn_config *cfg, const kvarn_cache *cache, int first_block,
                      int num_blocks, int rotated, float *k_out, float *v_out, void *stream);

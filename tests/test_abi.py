@@ -119,3 +119,14 @@ def test_dequantize_range_checked():
     L = kvarn.lib()
     assert L.kvarn_dequantize(ctypes.byref(cfg), ctypes.byref(cs), 3, 2, 0, None, None, None) == kvarn.KVARN_EINVAL
     assert L.kvarn_dequantize(ctypes.byref(cfg), ctypes.byref(cs), -1, 1, 0, None, None, None) == kvarn.KVARN_EINVAL
+
+
+def test_grid_overflow_rejected_on_host():
+    """One CTA per (sequence, kv head, block): a call whose grid would not fit an int is refused."""
+    cfg = kvarn.Config(1 << 12, 1 << 12, 128, 1 << 20).c()  # 2^24 units
+    assert _call_quant(cfg, T=128 * 127) == kvarn.KVARN_EINVAL   # 2^24 x 128 CTAs
+    cs = kvarn.kvarn_cache(16, 32, 48, 64, 80, 96, 112)
+    L = kvarn.lib()
+    assert L.kvarn_dequantize(ctypes.byref(cfg), ctypes.byref(cs), 0, 128, 0, None, None, None) == kvarn.KVARN_EINVAL
+    assert L.kvarn_token_errors(ctypes.byref(cfg), ctypes.c_void_p(16), ctypes.c_void_p(32), 128 * 128, 0,
+                                ctypes.byref(cs), ctypes.c_void_p(48), ctypes.c_void_p(64), None) == kvarn.KVARN_EINVAL
