@@ -178,22 +178,47 @@ class KVCache:
             self.k_records, self.v_records, self.k_tail, self.v_tail, self.n_tokens, self.arrive, self.status)))
 
 
-def _need(t, name, dtype=None):
+def _need(t, name, dtype=None, shape=None):
+    """The C ABI takes bare pointers: dtype, shape and layout are checked here, before any launch
+    (the device is checked last, by _on_device, once every shape is known to be right)."""
     if t is None:
         raise ValueError(f"{name} is required")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
-    if not t.is_contiguous():
-        raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _on_device(**tensors):
+    for name, t in tensors.items():
+        if t is not None and not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def _need_cache(cfg: Config, cache: KVCache):
+    """The cache's buffers must have the sizes cfg implies (the kernels index them from cfg)."""
+    S, H, D, T = cfg.num_seqs, cfg.num_kv_heads, cfg.head_dim, cfg.block_tokens
+    rec = (S, H, cfg.max_blocks, record_bytes(cfg))
+    for name in ("k_records", "v_records"):
+        _need(getattr(cache, name), f"cache.{name}", torch.uint8, rec)
+    for name in ("k_tail", "v_tail"):
+        _need(getattr(cache, name), f"cache.{name}", cfg.torch_dtype, (S, H, T, D))
+    for name in ("n_tokens", "arrive"):
+        _need(getattr(cache, name), f"cache.{name}", torch.int32, (S,))
+    _need(cache.status, "cache.status", torch.int32, (1,))
 
 
 def quantize_blocks(cfg: Config, k, v, cache: KVCache, first_block: int = 0, debug: bool = False, stream=None):
     """kvarn_quantize_blocks: k, v [S, Hkv, T, D] -> records (+ tail).  Returns (debug_k, debug_v) if debug."""
-    _need(k, "k", cfg.torch_dtype)
-    _need(v, "v", cfg.torch_dtype)
+    if k is None or k.dim() != 4:
+        raise ValueError("k must be a 4-d tensor [S, Hkv, T, D]")
     T = k.shape[2]
+    _need(k, "k", cfg.torch_dtype, (cfg.num_seqs, cfg.num_kv_heads, T, cfg.head_dim))
+    _need(v, "v", cfg.torch_dtype, k.shape)
+    _need_cache(cfg, cache)
+    _on_device(k=k, v=v, cache=cache.k_records)
     dk = dv = None
     if debug:
         nb = T // cfg.block_tokens
@@ -208,8 +233,10 @@ def quantize_blocks(cfg: Config, k, v, cache: KVCache, first_block: int = 0, deb
 
 def append_token(cfg: Config, k, v, cache: KVCache, stream=None):
     """kvarn_append_token: k, v [S, Hkv, D]."""
-    _need(k, "k", cfg.torch_dtype)
-    _need(v, "v", cfg.torch_dtype)
+    _need(k, "k", cfg.torch_dtype, (cfg.num_seqs, cfg.num_kv_heads, cfg.head_dim))
+    _need(v, "v", cfg.torch_dtype, k.shape)
+    _need_cache(cfg, cache)
+    _on_device(k=k, v=v, cache=cache.k_records)
     c, cs = cfg.c(), cache.struct()
     _check(lib().kvarn_append_token(ctypes.byref(c), _ptr(k), _ptr(v), ctypes.byref(cs), _stream(stream)),
            "kvarn_append_token")
@@ -225,16 +252,20 @@ def decode_workspace(cfg: Config, num_q_heads: int, device="cuda"):
 def decode_attention(cfg: Config, q, cache: KVCache, max_tokens: int, out=None, workspace=None,
                      softmax_scale: float = 0.0, stream=None):
     """kvarn_decode_attention: q [S, Hq, D] -> out [S, Hq, D] fp32."""
-    _need(q, "q", cfg.torch_dtype)
+    if q is None or q.dim() != 3:
+        raise ValueError("q must be a 3-d tensor [S, Hq, D]")
     Hq = q.shape[1]
+    _need(q, "q", cfg.torch_dtype, (cfg.num_seqs, Hq, cfg.head_dim))
+    _need_cache(cfg, cache)
     if out is None:
         out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
-    _need(out, "out", torch.float32)
+    _need(out, "out", torch.float32, q.shape)
+    _on_device(q=q, out=out, cache=cache.k_records, workspace=workspace)
     if workspace is None:
         workspace = decode_workspace(cfg, Hq, q.device)
     c, cs = cfg.c(), cache.struct()
     _check(lib().kvarn_decode_attention(ctypes.byref(c), _ptr(q), int(Hq), float(softmax_scale), ctypes.byref(cs),
-                                        int(max_tokens), _ptr(out), _ptr(workspace), int(workspace.numel()),
+                                        int(max_tokens), _ptr(out), _ptr(workspace), int(workspace.numel() * workspace.element_size()),
                                         _stream(stream)), "kvarn_decode_attention")
     return out
 
@@ -244,8 +275,12 @@ def decode_attention_noalloc(cfg: Config, q, cache: KVCache, max_tokens: int, ou
     """kvarn_decode_attention_noalloc: like decode_attention, with the library's own static workspace.
 
     `out` must be given (this path allocates nothing); calls that overlap on the GPU race."""
-    _need(q, "q", cfg.torch_dtype)
-    _need(out, "out", torch.float32)
+    if q is None or q.dim() != 3:
+        raise ValueError("q must be a 3-d tensor [S, Hq, D]")
+    _need(q, "q", cfg.torch_dtype, (cfg.num_seqs, q.shape[1], cfg.head_dim))
+    _need(out, "out", torch.float32, q.shape)
+    _need_cache(cfg, cache)
+    _on_device(q=q, out=out, cache=cache.k_records)
     c, cs = cfg.c(), cache.struct()
     _check(lib().kvarn_decode_attention_noalloc(ctypes.byref(c), _ptr(q), int(q.shape[1]), float(softmax_scale),
                                                 ctypes.byref(cs), int(max_tokens), _ptr(out), _stream(stream)),
@@ -256,17 +291,21 @@ def decode_attention_noalloc(cfg: Config, q, cache: KVCache, max_tokens: int, ou
 def decode_attention_multi(cfg: Config, q, cache: KVCache, max_tokens: int, out=None, workspace=None,
                            softmax_scale: float = 0.0, stream=None):
     """kvarn_decode_attention_multi: q [S, Q, Hq, D] (the last Q tokens of each sequence) -> out fp32, same shape."""
-    _need(q, "q", cfg.torch_dtype)
+    if q is None or q.dim() != 4:
+        raise ValueError("q must be a 4-d tensor [S, Q, Hq, D]")
     S, Q, Hq, D = q.shape
+    _need(q, "q", cfg.torch_dtype, (cfg.num_seqs, Q, Hq, cfg.head_dim))
+    _need_cache(cfg, cache)
     if out is None:
         out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
-    _need(out, "out", torch.float32)
+    _need(out, "out", torch.float32, q.shape)
+    _on_device(q=q, out=out, cache=cache.k_records, workspace=workspace)
     if workspace is None:
         workspace = decode_workspace(cfg, Q * Hq, q.device)
     c, cs = cfg.c(), cache.struct()
     _check(lib().kvarn_decode_attention_multi(ctypes.byref(c), _ptr(q), int(Hq), int(Q), float(softmax_scale),
                                               ctypes.byref(cs), int(max_tokens), _ptr(out), _ptr(workspace),
-                                              int(workspace.numel()), _stream(stream)),
+                                              int(workspace.numel() * workspace.element_size()), _stream(stream)),
            "kvarn_decode_attention_multi")
     return out
 
@@ -274,13 +313,17 @@ def decode_attention_multi(cfg: Config, q, cache: KVCache, max_tokens: int, out=
 def decode_selftest_timeout(cfg: Config, q, cache: KVCache, max_tokens: int, stream=None):
     """kvarn_decode_selftest_timeout: decode with every first K copy withheld and 1 ms waits; returns the output
     (not meaningful) -- the caller checks KVARN_STATUS_TIMEOUT in cache.status."""
-    _need(q, "q", cfg.torch_dtype)
+    if q is None or q.dim() != 3:
+        raise ValueError("q must be a 3-d tensor [S, Hq, D]")
     Hq = q.shape[1]
+    _need(q, "q", cfg.torch_dtype, (cfg.num_seqs, Hq, cfg.head_dim))
+    _need_cache(cfg, cache)
+    _on_device(q=q, cache=cache.k_records)
     out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
     workspace = decode_workspace(cfg, Hq, q.device)
     c, cs = cfg.c(), cache.struct()
     _check(lib().kvarn_decode_selftest_timeout(ctypes.byref(c), _ptr(q), int(Hq), ctypes.byref(cs), int(max_tokens),
-                                               _ptr(out), _ptr(workspace), int(workspace.numel()), _stream(stream)),
+                                               _ptr(out), _ptr(workspace), int(workspace.numel() * workspace.element_size()), _stream(stream)),
            "kvarn_decode_selftest_timeout")
     return out
 
@@ -288,7 +331,13 @@ def decode_selftest_timeout(cfg: Config, q, cache: KVCache, max_tokens: int, str
 def token_errors(cfg: Config, k, v, cache: KVCache, first_block: int = 0, stream=None):
     """kvarn_token_errors -> (err_k, err_v) fp32 [S, Hkv, T_total, 2]: per token (|‖x^‖/‖x‖ - 1|, 1 - cos)
     of the records from first_block on against the original rows k, v [S, Hkv, T_total, D]."""
+    if k is None or k.dim() != 4:
+        raise ValueError("k must be a 4-d tensor [S, Hkv, T, D]")
     n = k.shape[2]
+    _need(k, "k", cfg.torch_dtype, (cfg.num_seqs, cfg.num_kv_heads, n, cfg.head_dim))
+    _need(v, "v", cfg.torch_dtype, k.shape)
+    _need_cache(cfg, cache)
+    _on_device(k=k, v=v, cache=cache.k_records)
     ek = torch.empty(k.shape[0], k.shape[1], n, 2, dtype=torch.float32, device=k.device)
     ev = torch.empty_like(ek)
     c, cs = cfg.c(), cache.struct()
@@ -299,6 +348,8 @@ def token_errors(cfg: Config, k, v, cache: KVCache, first_block: int = 0, stream
 
 def dequantize(cfg: Config, cache: KVCache, first_block: int, num_blocks: int, rotated: bool = False, stream=None):
     """kvarn_dequantize -> (k_out, v_out) fp32 [S, Hkv, num_blocks*T, D]."""
+    _need_cache(cfg, cache)
+    _on_device(cache=cache.k_records)
     shape = (cfg.num_seqs, cfg.num_kv_heads, num_blocks * cfg.block_tokens, cfg.head_dim)
     ko = torch.empty(shape, dtype=torch.float32, device=cache.k_records.device)
     vo = torch.empty_like(ko)

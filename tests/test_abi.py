@@ -130,3 +130,37 @@ def test_grid_overflow_rejected_on_host():
     assert L.kvarn_dequantize(ctypes.byref(cfg), ctypes.byref(cs), 0, 128, 0, None, None, None) == kvarn.KVARN_EINVAL
     assert L.kvarn_token_errors(ctypes.byref(cfg), ctypes.c_void_p(16), ctypes.c_void_p(32), 128 * 128, 0,
                                 ctypes.byref(cs), ctypes.c_void_p(48), ctypes.c_void_p(64), None) == kvarn.KVARN_EINVAL
+
+
+def test_binding_checks_shapes_before_launch():
+    """The binding refuses tensors whose shape, dtype or cache sizes do not follow the config, on the host."""
+    import torch
+    cfg = kvarn.Config(2, 2, 128, 4)
+    cache = kvarn.KVCache(cfg, device="cpu")
+    k = torch.zeros(2, 2, 256, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="shape"):
+        kvarn.quantize_blocks(cfg, k[:, :, :, :64].contiguous(), k[:, :, :, :64].contiguous(), cache)
+    with pytest.raises(ValueError, match="shape"):
+        kvarn.quantize_blocks(cfg, k, k[:1].contiguous(), cache)
+    with pytest.raises(ValueError, match="bfloat16"):
+        kvarn.quantize_blocks(cfg, k.float(), k.float(), cache)
+    with pytest.raises(ValueError, match="contiguous"):
+        kvarn.quantize_blocks(cfg, k.transpose(1, 0), k.transpose(1, 0), cache)
+    with pytest.raises(ValueError, match="CUDA"):  # well-formed, but not on the device
+        kvarn.quantize_blocks(cfg, k, k, cache)
+    other = kvarn.KVCache(kvarn.Config(2, 2, 128, 8), device="cpu")  # more blocks than cfg says
+    with pytest.raises(ValueError, match="cache.k_records"):
+        kvarn.quantize_blocks(cfg, k, k, other)
+    with pytest.raises(ValueError, match="shape"):
+        kvarn.append_token(cfg, k[:, :, 0, :96].contiguous(), k[:, :, 0, :96].contiguous(), cache)
+    q = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="shape"):
+        kvarn.decode_attention(cfg, q, cache, 256, out=torch.zeros(2, 8, 64))
+    with pytest.raises(ValueError, match="shape"):
+        kvarn.decode_attention(cfg, q[:1].contiguous(), cache, 256)
+    with pytest.raises(ValueError, match="4-d"):
+        kvarn.decode_attention_multi(cfg, q, cache, 256)
+    with pytest.raises(ValueError, match="shape"):
+        kvarn.token_errors(cfg, k, k[:, :, :128].contiguous(), cache)
+    with pytest.raises(ValueError, match="cache.k_tail"):
+        kvarn.dequantize(kvarn.Config(2, 2, 128, 4, dtype=kvarn.KVARN_F32), cache, 0, 1)
