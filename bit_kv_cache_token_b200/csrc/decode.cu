@@ -1,4 +1,5 @@
-// decode.cu -- single-token decode attention over the packed 2-bit cache.
+// decode.cu -- decode attention (one or a few query tokens per sequence) over
+// the packed 2-bit cache.
 //
 // KVarN decode (abstract: attention over the 2-bit cache in long-horizon
 // decoding; rndamp.com article, "Numbers": the second scale is fused into the
