@@ -133,6 +133,21 @@ def test_append_capacity_sets_status_and_stops():
     assert int(cache.status.item()) & kvarn.KVARN_STATUS_CAPACITY
 
 
+def test_scale_beyond_binary16_sets_nonfinite_status():
+    """Token scales r_t near 1e6 exceed the binary16 range (65504): the quantiser flags the status word."""
+    S, H, D = 1, 1, 128
+    cfg = _cfg(S, H, D, 1, torch.float32, 128)
+    cache = kvarn.KVCache(cfg)
+    k, v = _inputs(S, H, D, 128, torch.float32, 4, 0.5, None, 15)
+    kd, vd = k.to(DEV), v.to(DEV)
+    kvarn.quantize_blocks(cfg, kd, vd, cache)
+    torch.cuda.synchronize()
+    assert int(cache.status.item()) == 0
+    kvarn.quantize_blocks(cfg, (kd * 1e6).contiguous(), vd, cache)
+    torch.cuda.synchronize()
+    assert int(cache.status.item()) & kvarn.KVARN_STATUS_NONFINITE
+
+
 def _oracle_cache(cfg, k, v, L, hb, sweeps=4):
     """Fill a GPU cache with ORACLE-packed records and the raw tail; return (cache, krec, vrec) numpy."""
     S, H, D = cfg.num_seqs, cfg.num_kv_heads, cfg.head_dim
