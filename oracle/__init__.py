@@ -8,7 +8,7 @@ The arithmetic lives in ``kvarn_oracle.c`` (plain C, fp64, explicit
 definitions).  This module only loads the shared object and marshals numpy
 arrays.  Sources: the paper "KVarN: Variance-Normalized KV-Cache Quantization
 Mitigates Error Accumulation in Reasoning Tasks" -- abstract (Hadamard
-rotation, dual-scaling variance normalisation across both axes of K and V,
+rotation, then a variance normalisation with a token scale and a channel scale for K and V,
 2-bit), and the rndamp.com article, section "How It Works" items 1-2 and
 section "Numbers" (the second scale fused into dequantisation).
 """

@@ -8,9 +8,9 @@
  *
  * Sources (web pages about the paper "KVarN: Variance-Normalized KV-Cache
  * Quantization Mitigates Error Accumulation in Reasoning Tasks"):
- *   [abs]  codewithpapers.app paper record, abstract: Hadamard rotation, then
- *          dual-scaling variance normalisation across both axes of the K and V
- *          matrices, then 2-bit quantisation.
+ *   [abs]  codewithpapers.app paper record, abstract: a Hadamard rotation, then
+ *          a variance normalisation with two scales, one along the token axis
+ *          and one along the channel axis, of K and of V, then 2-bit codes.
  *   [how]  rndamp.com article, section "How It Works", item 1 (Hadamard
  *          transform in the channel dimension, O(N log N) online) and item 2
  *          (iterative algorithm balancing the rows and columns so that the
@@ -79,16 +79,26 @@ void kvo_rotate(const double *x, int D, int hb, double *y)
 /* Dual-axis variance normalisation [how, item 2; abs]                 */
 /* ------------------------------------------------------------------ */
 
-/* Population standard deviation of n values; a zero variance gives 1. */
-static double kvo_std_or_one(const double *z, int n)
+/*
+ * Population standard deviation of n values, or 0 when their variance is
+ * zero.  The variance does not change when every value is shifted by the
+ * same amount, so it is taken of z_i - z_0 (two passes: mean, then the mean
+ * square deviation).  The shift makes a constant sequence give exactly
+ * zero, whatever rounding the mean of equal values would carry.
+ */
+static double kvo_std_or_zero(const double *z, int n)
 {
+    const double z0 = z[0];
     double mean = 0.0;
-    for (int i = 0; i < n; ++i) mean += z[i];
+    for (int i = 0; i < n; ++i) mean += z[i] - z0;
     mean /= (double)n;
     double var = 0.0;
-    for (int i = 0; i < n; ++i) var += (z[i] - mean) * (z[i] - mean);
+    for (int i = 0; i < n; ++i) {
+        const double e = (z[i] - z0) - mean;
+        var += e * e;
+    }
     var /= (double)n;
-    return var > 0.0 ? sqrt(var) : 1.0;
+    return var > 0.0 ? sqrt(var) : 0.0;
 }
 
 /*
@@ -96,9 +106,20 @@ static double kvo_std_or_one(const double *z, int n)
  * Start from c = 1.  Each sweep first sets every row scale
  *     r_t = std_d( X[t][d] / c[d] ),
  * then every column scale
- *     c_d = std_t( X[t][d] / r[t] ).
- * After the last sweep every column of X / (r c) has variance exactly 1 and
- * the row variances are close to uniform.  sweeps == 0 leaves r = c = 1.
+ *     c_d = std_t( X[t][d] / r[t] ),
+ * then moves the common factor of the channel scales into the token scales:
+ *     g = geometric mean of c,  c_d <- c_d / g,  r_t <- r_t * g.
+ * Only the products r_t c_d enter Y = X / (r c), and they are unchanged by
+ * the last step; without it a block whose tokens share a large common part
+ * lets r grow and c shrink by the same factor every sweep, far outside the
+ * binary16 range the scales are stored in.
+ * A row or column whose variance is zero carries no scale information: it
+ * takes scale 1 and stays out of the gauge step (g is the geometric mean of
+ * the other channel scales, 1 if there are none; such rows are not
+ * multiplied by g).
+ * After the last sweep every column of X / (r c) with nonzero variance has
+ * variance exactly 1, the row variances are close to uniform and the channel
+ * scales have geometric mean 1.  sweeps == 0 leaves r = c = 1.
  */
 void kvo_normalize(const double *X, int T, int D, int sweeps, double *r, double *c)
 {
@@ -108,12 +129,19 @@ void kvo_normalize(const double *X, int T, int D, int sweeps, double *r, double 
     for (int k = 0; k < sweeps; ++k) {
         for (int t = 0; t < T; ++t) {
             for (int d = 0; d < D; ++d) z[d] = X[(size_t)t * D + d] / c[d];
-            r[t] = kvo_std_or_one(z, D);
+            r[t] = kvo_std_or_zero(z, D);          /* 0 marks a zero-variance row */
         }
         for (int d = 0; d < D; ++d) {
-            for (int t = 0; t < T; ++t) z[t] = X[(size_t)t * D + d] / r[t];
-            c[d] = kvo_std_or_one(z, T);
+            for (int t = 0; t < T; ++t) z[t] = X[(size_t)t * D + d] / (r[t] > 0.0 ? r[t] : 1.0);
+            c[d] = kvo_std_or_zero(z, T);          /* 0 marks a zero-variance column */
         }
+        double lsum = 0.0;
+        int n = 0;
+        for (int d = 0; d < D; ++d)
+            if (c[d] > 0.0) { lsum += log(c[d]); ++n; }
+        const double g = n > 0 ? exp(lsum / (double)n) : 1.0;
+        for (int d = 0; d < D; ++d) c[d] = c[d] > 0.0 ? c[d] / g : 1.0;
+        for (int t = 0; t < T; ++t) r[t] = r[t] > 0.0 ? r[t] * g : 1.0;
     }
     free(z);
 }
@@ -131,7 +159,8 @@ void kvo_normalize(const double *X, int T, int D, int sweeps, double *r, double 
  *   codes (T x D)   2-bit codes 0..3, one per byte (unpacked)
  * Y = Xrot / (r_t c_d) with the unrounded scales; within each group
  * m = min Y, s = (max Y - m) / 3, code = clamp(rint((Y - m) / s), 0, 3), and
- * a group with s == 0 gets code 0 everywhere.
+ * a group with s == 0 gets code 0 everywhere.  The returned r includes the
+ * token gauge described below.
  */
 void kvo_quantize_block(const double *X, int T, int D, int hb, int sweeps, int G,
                         double *Xrot, double *r, double *c, double *s, double *m,
@@ -145,11 +174,27 @@ void kvo_quantize_block(const double *X, int T, int D, int hb, int sweeps, int G
     const int ng = D / G;
     double *y = (double *)malloc(sizeof(double) * (size_t)G);
     for (int t = 0; t < T; ++t) {
+        /* Token gauge: r_t times (s, m) of the token is what dequantises, so a
+         * power of two can move between them exactly.  When the token's
+         * largest |Y| reaches 2^14, 2^k (k = floor(log2 max|Y|) - 13) moves
+         * into r_t, which brings max|Y| into [2^13, 2^14) and keeps s and m
+         * inside binary16; Y / 2^k is exact and the codes do not change. */
+        double ymax = 0.0;
+        for (int d = 0; d < D; ++d) {
+            const double a = fabs(xr[(size_t)t * D + d] / (r[t] * c[d]));
+            if (a > ymax) ymax = a;
+        }
+        double tg = 1.0;
+        if (ymax >= 16384.0) {
+            int e2;
+            (void)frexp(ymax, &e2);                 /* ymax = f * 2^e2, f in [0.5, 1) */
+            tg = ldexp(1.0, (e2 - 1) - 13);
+        }
         for (int g = 0; g < ng; ++g) {
             double lo = INFINITY, hi = -INFINITY;
             for (int i = 0; i < G; ++i) {
                 const int d = g * G + i;
-                y[i] = xr[(size_t)t * D + d] / (r[t] * c[d]);
+                y[i] = xr[(size_t)t * D + d] / (r[t] * c[d]) / tg;
                 if (y[i] < lo) lo = y[i];
                 if (y[i] > hi) hi = y[i];
             }
@@ -171,6 +216,7 @@ void kvo_quantize_block(const double *X, int T, int D, int hb, int sweeps, int G
                 codes[e] = (uint8_t)q;
             }
         }
+        r[t] *= tg;
     }
     if (Xrot) memcpy(Xrot, xr, sizeof(double) * (size_t)T * D);
     free(y);

@@ -5,7 +5,7 @@ Accumulation in Reasoning Tasks" -- abstract (Hadamard rotation, dual-scaling
 variance normalisation over both axes, 2-bit) and the rndamp.com article,
 "How It Works" items 1-2, "Numbers" (second scale fused into dequantisation).
 The pages print no worked example, so the pins are closed forms, invariants,
-library routines and brute force (see tests/golden/README.md).
+library routines and brute force.
 """
 import math
 
@@ -87,13 +87,15 @@ def _paired_rank_one(T=16, D=64, seed=3):
 @pytest.mark.parametrize("sweeps", [1, 2, 4])
 def test_closed_form_paired_rank_one(sweeps):
     """X_td = a_t b_d (-1)^(t+d), a and b positive and paired, rotation off:
-    r_t = a_t RMS(b), c_d = b_d / RMS(b) after the first sweep and at every later one,
-    Y = +-1 and the codes are 0 / 3 by the sign pattern."""
+    r_t = a_t GM(b), c_d = b_d / GM(b) (GM = geometric mean) after the first sweep and at every later
+    one, Y = +-1 and the codes are 0 / 3 by the sign pattern.  Without the gauge step the split would
+    be r_t = a_t RMS(b), c_d = b_d / RMS(b): the product r_t c_d = a_t b_d is the same either way."""
     a, b, X = _paired_rank_one()
-    rms = math.sqrt(np.mean(b * b))
+    gm = math.exp(np.mean(np.log(b)))
     r, c = oracle.normalize(X, sweeps)
-    np.testing.assert_allclose(r, a * rms, rtol=1e-13)
-    np.testing.assert_allclose(c, b / rms, rtol=1e-13)
+    np.testing.assert_allclose(r, a * gm, rtol=1e-13)
+    np.testing.assert_allclose(c, b / gm, rtol=1e-13)
+    np.testing.assert_allclose(np.outer(r, c), np.outer(a, b), rtol=1e-13)
     q = oracle.quantize_block(X, hb=0, sweeps=sweeps, group=32)
     sign = (-1.0) ** np.add.outer(np.arange(16), np.arange(64))
     np.testing.assert_array_equal(q["codes"], np.where(sign > 0, 3, 0))
@@ -129,13 +131,106 @@ def test_power_of_two_token_scaling_is_exact(hb):
 
 
 def test_zero_rows_and_columns_get_unit_scale():
+    """A zero row or column has zero variance, takes scale 1 and stays out of the gauge step: the other channel
+    scales have geometric mean 1 on their own.  The zero row codes to 0 with s = m = 0."""
     X = np.random.default_rng(2).standard_normal((128, 64))
     X[3] = 0.0
     X[:, 10] = 0.0
     r, c = oracle.normalize(X, 4)
     assert r[3] == 1.0 and c[10] == 1.0
+    assert abs(np.mean(np.log(np.delete(c, 10)))) < 1e-14
     q = oracle.quantize_block(X, hb=0, sweeps=4)
-    assert np.all(q["codes"][3] == 0) and np.all(q["s"][3] == 0.0)
+    assert np.all(q["codes"][3] == 0) and np.all(q["s"][3] == 0.0) and np.all(q["m"][3] == 0.0)
+
+
+def _population_std(x):
+    return float(np.sqrt(np.mean((x - x.mean()) ** 2)))
+
+
+@pytest.mark.parametrize("hb", [0, 128])
+def test_identical_tokens_give_token_std_and_unit_channel_scales(hb):
+    """128 copies of one token: every column of X / r is constant, so every c_d = 1 exactly (zero variance, and
+    the gauge of all-ones is 1) and r_t is the population std of the rotated token.  Scaling copies by powers of
+    two scales their r_t by the same power and leaves c = 1."""
+    x = np.random.default_rng(12).standard_normal(128) * np.exp(np.random.default_rng(13).standard_normal(128))
+    X = np.tile(x, (128, 1))
+    q = oracle.quantize_block(X, hb=hb, sweeps=4)
+    np.testing.assert_array_equal(q["c"], np.ones(128))
+    np.testing.assert_allclose(q["r"], _population_std(oracle.rotate(x, hb)), rtol=1e-14)
+    p = 2.0 ** np.random.default_rng(14).integers(-6, 7, size=128)
+    q2 = oracle.quantize_block(X * p[:, None], hb=hb, sweeps=4)
+    np.testing.assert_array_equal(q2["c"], np.ones(128))
+    np.testing.assert_array_equal(q2["r"], q["r"] * p)
+    np.testing.assert_array_equal(q2["codes"], q["codes"])
+
+
+def _common_component_blocks():
+    """Blocks whose tokens share a large common part: near-identical tokens, and a DC offset on one channel."""
+    rng = np.random.default_rng(15)
+    x = rng.standard_normal(128) * np.exp(rng.standard_normal(128))
+    base = rng.standard_normal((128, 128))
+    out = [("identical+1e-2", np.tile(x, (128, 1)) + 1e-2 * base),
+           ("identical+1e-4", np.tile(x, (128, 1)) + 1e-4 * base)]
+    for off in (100.0, 1000.0):
+        for ch in (0, 77):
+            X = base.copy()
+            X[:, ch] += off
+            out.append((f"dc{off:g}@{ch}", X))
+    return out
+
+
+@pytest.mark.parametrize("hb", [0, 128])
+def test_common_component_keeps_scales_in_binary16(hb):
+    """On blocks with a large common token component every stored scale (r, c, s, m) is a finite, nonzero (r, c)
+    binary16 number -- the iteration without the gauge step drives r and c to 1e7..1e14 and 1e-10..1e-19 on these
+    blocks -- the channel scales have geometric mean 1, the columns of Y = X / (r c) have unit variance, and no
+    stored |Y| reaches 2^14."""
+    for name, X in _common_component_blocks():
+        Xb = oracle.rotate(X, hb)
+        r, c = oracle.normalize(Xb, 4)
+        assert abs(np.mean(np.log(c))) < 1e-13, name
+        np.testing.assert_allclose((Xb / (r[:, None] * c[None, :])).var(axis=0), 1.0, rtol=0, atol=1e-9, err_msg=name)
+        q = oracle.quantize_block(X, hb=hb, sweeps=4)
+        for key in ("r", "c", "s", "m"):
+            h = np.array([oracle.f16_value(oracle.f16_bits(v)) for v in np.ravel(q[key])])
+            assert np.all(np.isfinite(h)), (name, key, np.abs(q[key]).max())
+            if key in ("r", "c"):
+                assert np.all(h > 0), (name, key, q[key].min())
+        Ys = q["xrot"] / (q["r"][:, None] * q["c"][None, :])
+        assert np.abs(Ys).max() < 2.0 ** 14, name
+
+
+@pytest.mark.parametrize("A,k", [(1000.0, 0), (100000.0, 3), (3.0e6, 8)])
+def test_token_gauge_closed_form(A, k):
+    """X_td = A + (-1)^(t+d), rotation off: r = c = 1 exactly (every row and column is A +- 1), so Y = X.  Once
+    max |Y| = A + 1 reaches 2^14 the token gauge moves 2^k, k = floor(log2(A + 1)) - 13, into every r_t: r = 2^k,
+    m = (A - 1) / 2^k, s = 2 / (3 2^k), and the codes stay 3 / 0 by the sign pattern."""
+    sign = (-1.0) ** np.add.outer(np.arange(128), np.arange(64))
+    X = A + sign
+    r, c = oracle.normalize(X, 4)
+    np.testing.assert_array_equal(r, np.ones(128))
+    np.testing.assert_array_equal(c, np.ones(64))
+    q = oracle.quantize_block(X, hb=0, sweeps=4)
+    assert k == max(0, math.floor(math.log2(A + 1)) - 13)
+    np.testing.assert_array_equal(q["r"], np.full(128, 2.0 ** k))
+    np.testing.assert_array_equal(q["c"], np.ones(64))
+    np.testing.assert_array_equal(q["m"], np.full((128, 2), (A - 1) / 2.0 ** k))
+    np.testing.assert_allclose(q["s"], 2.0 / (3 * 2.0 ** k), rtol=1e-15)
+    np.testing.assert_array_equal(q["codes"], np.where(sign > 0, 3, 0))
+
+
+def test_gauge_moves_only_a_common_factor():
+    """Against the iteration written without the gauge step (a plain numpy loop, central variance): the products
+    r_t c_d agree and the gauged channel scales are the ungauged ones divided by their geometric mean."""
+    X, _ = _config0_k(4)
+    Xb = oracle.rotate(X[:128], 64)
+    c0 = np.ones(64)
+    for _ in range(4):
+        r0 = (Xb / c0).std(axis=1)
+        c0 = (Xb / r0[:, None]).std(axis=0)
+    r, c = oracle.normalize(Xb, 4)
+    np.testing.assert_allclose(np.outer(r, c), np.outer(r0, c0), rtol=1e-12)
+    np.testing.assert_allclose(c, c0 / math.exp(np.mean(np.log(c0))), rtol=1e-12)
 
 
 def test_zero_sweeps_is_plain_group_rtn():
