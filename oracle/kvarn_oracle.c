@@ -80,11 +80,20 @@ void kvo_rotate(const double *x, int D, int hb, double *y)
 /* ------------------------------------------------------------------ */
 
 /*
+ * A variance at most this fraction of the mean square counts as zero: the
+ * values agree to about 2^-20 of their size, below what the scales can
+ * resolve (a difference that small only arises from rounding, and whether
+ * it survives depends on the working precision, not on the data).
+ */
+#define KVO_ZERO_VAR_REL 0x1p-40
+
+/*
  * Population standard deviation of n values, or 0 when their variance is
- * zero.  The variance does not change when every value is shifted by the
- * same amount, so it is taken of z_i - z_0 (two passes: mean, then the mean
- * square deviation).  The shift makes a constant sequence give exactly
- * zero, whatever rounding the mean of equal values would carry.
+ * zero (KVO_ZERO_VAR_REL).  The variance does not change when every value
+ * is shifted by the same amount, so it is taken of z_i - z_0 (two passes:
+ * mean, then the mean square deviation).  The shift makes a constant
+ * sequence give exactly zero, whatever rounding the mean of equal values
+ * would carry.
  */
 static double kvo_std_or_zero(const double *z, int n)
 {
@@ -98,7 +107,8 @@ static double kvo_std_or_zero(const double *z, int n)
         var += e * e;
     }
     var /= (double)n;
-    return var > 0.0 ? sqrt(var) : 0.0;
+    const double mz = z0 + mean;             /* mean of the values */
+    return var > KVO_ZERO_VAR_REL * (var + mz * mz) ? sqrt(var) : 0.0;
 }
 
 /*
