@@ -7,9 +7,14 @@
 //      computed as a fast Walsh-Hadamard transform (O(N log N));
 //   2. dual-axis variance normalisation: starting from c = 1, each sweep sets
 //      r_t = std_d(X/c) for every token, then c_d = std_t(X/r) for every channel
-//      (population std; a zero variance gives scale 1);
+//      (population std), then divides c by g, the geometric mean of the channel
+//      scales, and multiplies r by g (only r_t c_d enters Y, and the split
+//      between the two is otherwise free to drift out of binary16); a row or
+//      column with zero variance takes scale 1 and stays out of the gauge;
 //   3. Y = X / (r c); per token and group of 32 channels: m = min Y,
 //      s = (max Y - m)/3, code = rint((Y - m)/s) in 0..3 (s = 0 -> code 0);
+//      a token whose largest |Y| reaches 2^14 moves a power of two from its
+//      (s, m) into r_t (token gauge, exact);
 //   4. store codes, binary16 (s, m), r and c in one block record.
 //
 // Thread layout (D threads = D/32 warps; warp j owns channel group j):
@@ -35,9 +40,18 @@ struct QuantSmem {
         float4 col[W][32][16];                 // column-sum transpose [warp][lane][chunk]
         unsigned char rec[Record<D>::kBytes];  // record staging
     } u;
-    float2 part[2][W][kBlockTokens];           // per-token partial (sum, sum of squares)
+    float part[2][W][kBlockTokens];            // per-token partial row sums: [0] of z, [1] of (z - mean)^2
     float ubuf[D];                             // 1 / c broadcast
+    float kbuf[D];                             // column shifts z[0][d]
+    float2 gpart[W];                           // per-warp (sum of log2 c, count) of nonzero-variance channels
+    float ymax[W][kBlockTokens];               // per-(group, token) largest |Y| (token gauge)
 };
+
+// A variance at most this fraction of the mean square counts as zero.  In
+// fp32, values that are all equal leave a residual of order 2^-48 of their
+// mean square through the fused shifts and sums; spreads of real data (bf16
+// or fp32 inputs, rotated) sit far above 2^-40.
+constexpr float kZeroVarRel = 9.094947e-13f;  // 2^-40
 
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, f2(-1.f, -1.f), a); }
 
@@ -144,8 +158,9 @@ __device__ __forceinline__ void rotate_block(float2 (&X)[4][16], QuantSmem<D> &s
 }
 
 // Quantise the block held in X (destroyed) into rec_out (global, 16-byte
-// aligned, Record<D>::kBytes); TENSOR 0 = K code order, 1 = V code order.  dbg: NULL or fp32 [T + D + 2*T*D/32] unrounded
-// r, c, s, m.  All D threads of the CTA must call this.
+// aligned, Record<D>::kBytes); TENSOR 0 = K code order, 1 = V code order.
+// dbg: NULL or fp32 [T + D + 2*T*D/32] unrounded r, c, s, m (as stored, token
+// gauge included).  All D threads of the CTA must call this.
 template <int D, int HB, int TENSOR>
 __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
                                unsigned char *__restrict__ rec_out, float *__restrict__ dbg,
@@ -159,82 +174,132 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
     rotate_block<D, HB>(X, sm);
 
     // ---- 2. dual-axis variance normalisation ------------------------------
+    // Rows: two passes (mean, then mean square deviation) over the D channels,
+    // whose partial sums cross the warps through shared memory.  Columns: one
+    // pass over the 128 tokens on values shifted by token 0's (lane 0's) z,
+    // whose partials cross the lanes through a shared-memory transpose.  Then
+    // the gauge: g = geometric mean of the nonzero-variance channel scales,
+    // c <- c / g (1 for a zero-variance column), r <- r g at the end.
     float2 u[16];  // 1 / c for this thread's 32 channels
 #pragma unroll
     for (int k = 0; k < 16; ++k) u[k] = f2(1.f, 1.f);
     float w[4] = {1.f, 1.f, 1.f, 1.f};    // 1 / r for this thread's 4 tokens
-    float rt[4] = {1.f, 1.f, 1.f, 1.f};   // r for this thread's 4 tokens
-    float cd = 1.f;                       // c of channel 32j + l (lane-owned)
+    float rt[4] = {1.f, 1.f, 1.f, 1.f};   // r for this thread's 4 tokens (0 marks zero variance)
+    float cd = 1.f;                       // c of channel 32j + l (lane-owned, gauged)
+    float g = 1.f;                        // gauge factor of the last column step
 
     for (int sw = 0; sw < sweeps; ++sw) {
-        // row step: r_t = std over the D channels of X / c
+        // row step, pass 1: mean over the D channels of z = X u
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-            float2 s1 = f2(0.f, 0.f), s2 = f2(0.f, 0.f);
-            if (sw == 0) {  // c = 1: X / c is X
+            float2 s1 = f2(0.f, 0.f), s1b = f2(0.f, 0.f);
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    s1 = __fadd2_rn(s1, X[r][k]);
-                    s2 = __ffma2_rn(X[r][k], X[r][k], s2);
-                }
-            } else {
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const float2 z = __fmul2_rn(X[r][k], u[k]);
-                    s1 = __fadd2_rn(s1, z);
-                    s2 = __ffma2_rn(z, z, s2);
-                }
+            for (int k = 0; k < 16; k += 2) {
+                s1 = __ffma2_rn(X[r][k], u[k], s1);
+                s1b = __ffma2_rn(X[r][k + 1], u[k + 1], s1b);
             }
-            sm.part[sw & 1][j][l + 32 * r] = f2(s1.x + s1.y, s2.x + s2.y);
+            s1 = __fadd2_rn(s1, s1b);
+            sm.part[0][j][l + 32 * r] = s1.x + s1.y;
+        }
+        __syncthreads();
+        float mean[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            float S1 = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < W; ++jj) S1 += sm.part[0][jj][l + 32 * r];
+            mean[r] = S1 * (1.f / D);
+        }
+        // row step, pass 2: mean square deviation from that mean
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const float2 nm = f2(-mean[r], -mean[r]);
+            float2 s2 = f2(0.f, 0.f), s2b = f2(0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < 16; k += 2) {
+                const float2 e = __ffma2_rn(X[r][k], u[k], nm);
+                const float2 eb = __ffma2_rn(X[r][k + 1], u[k + 1], nm);
+                s2 = __ffma2_rn(e, e, s2);
+                s2b = __ffma2_rn(eb, eb, s2b);
+            }
+            s2 = __fadd2_rn(s2, s2b);
+            sm.part[1][j][l + 32 * r] = s2.x + s2.y;
         }
         __syncthreads();
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-            float S1 = 0.f, S2 = 0.f;
+            float S2 = 0.f;
 #pragma unroll
-            for (int jj = 0; jj < W; ++jj) {
-                const float2 p = sm.part[sw & 1][jj][l + 32 * r];
-                S1 += p.x;
-                S2 += p.y;
-            }
-            const float mean = S1 * (1.f / D);
-            const float var = fmaf(-mean, mean, S2 * (1.f / D));
-            w[r] = var > 0.f ? rsqrtf(var) : 1.f;  // 1 / r_t
-            rt[r] = var > 0.f ? var * w[r] : 1.f;  // r_t = sqrt(var)
+            for (int jj = 0; jj < W; ++jj) S2 += sm.part[1][jj][l + 32 * r];
+            const float var = S2 * (1.f / D);
+            const bool nz = var > kZeroVarRel * fmaf(mean[r], mean[r], var);
+            const float is = rsqrtf(var);
+            w[r] = nz ? is : 1.f;         // 1 / r_t
+            rt[r] = nz ? var * is : 0.f;  // r_t = sqrt(var); 0 marks a zero-variance row (scale 1)
         }
-        // column step: c_d = std over the 128 tokens of X / r
+        // column step: c_d = std over the 128 tokens of z = X / r, on values
+        // shifted by token 0's z (lane 0, r = 0) for precision
+        if (l == 0) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float2 a = __fmul2_rn(X[0][2 * q], f2(w[0], w[0]));
+                const float2 b = __fmul2_rn(X[0][2 * q + 1], f2(w[0], w[0]));
+                reinterpret_cast<float4 *>(&sm.kbuf[32 * j])[q] = make_float4(a.x, a.y, b.x, b.y);
+            }
+        }
+        __syncwarp();
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const int k = 8 * half + kk;
+                const float2 kv = reinterpret_cast<const float2 *>(&sm.kbuf[32 * j])[k];
+                const float2 nk = f2(-kv.x, -kv.y);
                 float2 c1 = f2(0.f, 0.f), c2 = f2(0.f, 0.f);
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
-                    const float2 z = __fmul2_rn(X[r][k], f2(w[r], w[r]));
-                    c1 = __fadd2_rn(c1, z);
-                    c2 = __ffma2_rn(z, z, c2);
+                    const float2 e = __ffma2_rn(X[r][k], f2(w[r], w[r]), nk);
+                    c1 = __fadd2_rn(c1, e);
+                    c2 = __ffma2_rn(e, e, c2);
                 }
                 // chunk k of row l holds channels 2k, 2k+1 as (sum, sumsq) pairs
                 sm.u.col[j][l][k ^ (l & 15)] = make_float4(c1.x, c2.x, c1.y, c2.y);
             }
         }
         __syncwarp();
+        bool znz;  // this lane's channel has nonzero variance
         {
             // lane l sums column l (channel 32j + l) over the 32 rows
-            float2 acc = f2(0.f, 0.f);
+            float2 acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
             const int k = l >> 1, hi = l & 1;
 #pragma unroll
             for (int row = 0; row < 32; ++row) {
                 const float2 *chunk = reinterpret_cast<const float2 *>(&sm.u.col[j][row][k ^ (row & 15)]);
-                acc = __fadd2_rn(acc, chunk[hi]);
+                acc[row & 3] = __fadd2_rn(acc[row & 3], chunk[hi]);
             }
-            const float mean = acc.x * (1.f / kBlockTokens);
-            const float var = fmaf(-mean, mean, acc.y * (1.f / kBlockTokens));
-            const float ud = var > 0.f ? rsqrtf(var) : 1.f;  // 1 / c_d
-            cd = var > 0.f ? var * ud : 1.f;
-            __syncwarp();
-            sm.ubuf[32 * j + l] = ud;
+            const float2 tot = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+            const float me = tot.x * (1.f / kBlockTokens);  // mean of the shifted values
+            const float var = fmaf(-me, me, tot.y * (1.f / kBlockTokens));
+            const float mz = sm.kbuf[32 * j + l] + me;      // mean of z
+            znz = var > kZeroVarRel * fmaf(mz, mz, fmaxf(var, 0.f));
+            cd = znz ? sqrtf(var) : 1.f;
+            float lg = znz ? log2f(cd) : 0.f;
+            float cnt = znz ? 1.f : 0.f;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                lg += __shfl_xor_sync(0xffffffffu, lg, o);
+                cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+            }
+            if (l == 0) sm.gpart[j] = f2(lg, cnt);
+        }
+        __syncthreads();  // every warp's gauge partial is in
+        {
+            float2 tot = f2(0.f, 0.f);
+#pragma unroll
+            for (int jj = 0; jj < W; ++jj) tot = __fadd2_rn(tot, sm.gpart[jj]);
+            g = tot.y > 0.f ? exp2f(tot.x / tot.y) : 1.f;
+            cd = znz ? cd / g : 1.f;
+            sm.ubuf[32 * j + l] = 1.f / cd;
             __syncwarp();
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -243,6 +308,12 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
                 u[2 * q + 1] = f2(v.z, v.w);
             }
         }
+    }
+    // last gauge on the token scales: r <- r g (a zero-variance row keeps 1)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        rt[r] = rt[r] > 0.f ? rt[r] * g : 1.f;
+        w[r] = 1.f / rt[r];
     }
     __syncthreads();  // every warp is done with the shared transposes
 
@@ -256,6 +327,7 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
     // bit pattern is 0x4B400000 + code: multiply-adding the raw patterns with the
     // code weights and subtracting the pattern's share once packs them.
     uint32_t vacc[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // V: channel i in byte i%4 of vacc[i/4]
+    float gs[4], gm[4];  // this group's s and m in Y units, before the token gauge
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         const int t = l + 32 * r;
@@ -268,17 +340,20 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
             mx = max3(mx, z[k].x, z[k].y);
         }
         const float range = mx - mn;
-        // level = (Z - min) * 3 / range: Z = Y * r_t, so this equals (Y - m) / s
+        // level = (Z - min) * 3 / range: Z = Y * r_t, so this equals (Y - m) / s.
+        // Z - min is formed first: it lies in [0, range] whatever the offset of
+        // the group, so the level stays in [0, 3] and cannot spill into the
+        // neighbouring 2-bit fields of the packed words.
         const float kq = range > 0.f ? 3.f / range : 0.f;
         const float2 kq2 = f2(kq, kq);
-        const float2 nmk = f2(-mn * kq, -mn * kq);
+        const float2 mn2 = f2(mn, mn);
         // 12582912 = 1.5 * 2^23: adding it rounds the level to an integer
         // (ties to even) and leaves that integer in the low mantissa bits.
         const float2 magic = f2(12582912.f, 12582912.f);
         uint32_t kacc[4] = {0u, 0u, 0u, 0u};  // K: byte (tig, half) at bits 8*half of kacc[tig]
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-            const float2 lev = __fadd2_rn(__ffma2_rn(z[k], kq2, nmk), magic);
+            const float2 lev = __ffma2_rn(sub2(z[k], mn2), kq2, magic);
             const uint32_t b0 = __float_as_uint(lev.x), b1 = __float_as_uint(lev.y);
             // local channels 2k (b0) and 2k+1 (b1): x = k/4, tig = k%4
             if constexpr (TENSOR == 0) {
@@ -298,23 +373,9 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
                 rec[k_code_bit<D>(t, kch + 1) / 8] = (unsigned char)((v >> 8) & 0xFFu);
             }
         }
-        const float s = range * w[r] * (1.f / 3.f);
-        const float m = mn * w[r];
-        const __half hs = __float2half_rn(s), hm = __float2half_rn(m);
-        if (__hisinf(hs) || __hisnan(hs) || __hisinf(hm) || __hisnan(hm))
-            status_or(status, KVARN_STATUS_NONFINITE);
-        reinterpret_cast<__half *>(rec + R::kSOff)[t * (D / 32) + j] = hs;
-        reinterpret_cast<__half *>(rec + R::kMOff)[t * (D / 32) + j] = hm;
-        if (j == 0) {
-            const __half hr = __float2half_rn(rt[r]);
-            if (__hisinf(hr) || __hisnan(hr)) status_or(status, KVARN_STATUS_NONFINITE);
-            *reinterpret_cast<__half *>(rec + R::kROff + 2 * t) = hr;
-        }
-        if (dbg) {
-            if (j == 0) dbg[t] = rt[r];
-            dbg[kBlockTokens + D + t * (D / 32) + j] = s;
-            dbg[kBlockTokens + D + kBlockTokens * (D / 32) + t * (D / 32) + j] = m;
-        }
+        gs[r] = range * w[r] * (1.f / 3.f);
+        gm[r] = mn * w[r];
+        sm.ymax[j][t] = fmaxf(fabsf(mn), fabsf(mx)) * w[r];  // this group's largest |Y|
     }
     if constexpr (TENSOR == 1) {
         // each vacc word took 0x4B400000 * (1 + 4 + 16 + 64) * (1 + 256 + 65536 + 2^24)
@@ -324,6 +385,41 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
 #pragma unroll
         for (int i = 0; i < 32; ++i)
             rec[v_code_bit(l, 32 * j + i) / 8] = (unsigned char)(vacc[i >> 2] >> (8 * (i & 3)));
+    }
+    __syncthreads();  // every group's largest |Y| is in
+    // Token gauge: r_t times the token's (s, m) is what dequantises; when the
+    // token's largest |Y| reaches 2^14, the power of two 2^k with k =
+    // floor(log2 max|Y|) - 13 moves from (s, m) into r_t (exact: codes and
+    // products unchanged), which keeps s and m inside binary16.
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int t = l + 32 * r;
+        float ym = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < W; ++jj) ym = fmaxf(ym, sm.ymax[jj][t]);
+        float tg = 1.f, itg = 1.f;
+        if (ym >= 16384.f) {
+            const int e = (int)((__float_as_uint(ym) >> 23) & 0xFFu) - 127;  // floor(log2 ym)
+            tg = __uint_as_float((uint32_t)(e - 13 + 127) << 23);
+            itg = __uint_as_float((uint32_t)(127 - (e - 13)) << 23);
+        }
+        const float s = gs[r] * itg, m = gm[r] * itg;
+        const __half hs = __float2half_rn(s), hm = __float2half_rn(m);
+        if (__hisinf(hs) || __hisnan(hs) || __hisinf(hm) || __hisnan(hm))
+            status_or(status, KVARN_STATUS_NONFINITE);
+        reinterpret_cast<__half *>(rec + R::kSOff)[t * (D / 32) + j] = hs;
+        reinterpret_cast<__half *>(rec + R::kMOff)[t * (D / 32) + j] = hm;
+        const float rr = rt[r] * tg;
+        if (j == 0) {
+            const __half hr = __float2half_rn(rr);
+            if (__hisinf(hr) || __hisnan(hr)) status_or(status, KVARN_STATUS_NONFINITE);
+            *reinterpret_cast<__half *>(rec + R::kROff + 2 * t) = hr;
+        }
+        if (dbg) {
+            if (j == 0) dbg[t] = rr;
+            dbg[kBlockTokens + D + t * (D / 32) + j] = s;
+            dbg[kBlockTokens + D + kBlockTokens * (D / 32) + t * (D / 32) + j] = m;
+        }
     }
     {
         const __half hc = __float2half_rn(cd);

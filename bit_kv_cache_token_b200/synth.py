@@ -78,3 +78,32 @@ def layer_kv(seed: int, layer: int, num_seqs: int, num_kv_heads: int, num_tokens
     k = keys(base + 1 + 2 * first_position, f, num_seqs, num_tokens, sigma_k, first_position, dtype, device)
     v = values(base + 2 + 2 * first_position, num_seqs, num_kv_heads, num_tokens, head_dim, dtype, device)
     return k, v
+
+
+def common_component_kv(seed: int, kind: str, num_seqs: int, num_kv_heads: int, num_tokens: int, head_dim: int,
+                        amount: float, channel: int = 0, dtype=torch.bfloat16, device="cpu"):
+    """(K, V) whose tokens share a large common part, each [S, Hkv, T, D].
+
+    kind "identical": every token of a (sequence, kv head) is one random token x (N(0,1) times a lognormal(0,1)
+    channel factor) plus amount * N(0,1) per element (amount 0: exact copies).
+    kind "dc": N(0,1) per element with `amount` added to channel `channel` of every token.
+    kind "offset": `amount` + N(0,1) in every element (every row and column has mean/std = amount).
+    K and V use independent draws of the same recipe.
+    """
+    g = _gen(seed, device)
+    out = []
+    for _ in range(2):
+        shape = (num_seqs, num_kv_heads, num_tokens, head_dim)
+        if kind == "identical":
+            x = torch.randn(num_seqs, num_kv_heads, 1, head_dim, generator=g, device=device)
+            x = x * torch.exp(torch.randn(num_seqs, num_kv_heads, 1, head_dim, generator=g, device=device))
+            z = x.expand(shape) + amount * torch.randn(shape, generator=g, device=device)
+        elif kind == "dc":
+            z = torch.randn(shape, generator=g, device=device)
+            z[..., channel] += amount
+        elif kind == "offset":
+            z = amount + torch.randn(shape, generator=g, device=device)
+        else:
+            raise ValueError(kind)
+        out.append(z.contiguous().to(dtype))
+    return out[0], out[1]

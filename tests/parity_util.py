@@ -54,8 +54,9 @@ def view_record(rec, T: int, D: int, layout: int, G: int = 32) -> dict:
     return dict(codes=codes.astype(np.uint8), s=s.copy(), m=m.copy(), r=r.copy(), c=c.copy(), pad=pad.copy())
 
 
-def near_f16_midpoint(x) -> np.ndarray:
-    """True where x lies within 1e-5 relative of a binary16 rounding midpoint."""
+def near_f16_midpoint(x, window: float = None) -> np.ndarray:
+    """True where x lies within `window` (default 1e-5) relative of a binary16 rounding midpoint."""
+    window = WINDOW if window is None else window
     x = np.asarray(x, dtype=np.float64)
     h = x.astype(np.float16)
     bits = h.view(np.uint16).astype(np.int32)
@@ -64,22 +65,29 @@ def near_f16_midpoint(x) -> np.ndarray:
         nb = np.clip(bits + step * np.where(x < 0, -1, 1), 0, 0xFFFF).astype(np.uint16)
         nbv = nb.view(np.float16).astype(np.float64)
         mid = 0.5 * (h.astype(np.float64) + nbv)
-        out |= np.abs(x - mid) <= WINDOW * np.abs(x)
+        out |= np.abs(x - mid) <= window * np.abs(x)
     return out
 
 
-def near_boundary(v, s) -> np.ndarray:
+def near_boundary(v, s, window: float = None) -> np.ndarray:
+    window = WINDOW if window is None else window
     frac = np.asarray(v) - np.floor(v)
-    return (np.abs(frac - 0.5) < WINDOW) & (np.repeat(np.asarray(s), np.asarray(v).shape[-1] // np.asarray(s).shape[-1],
+    return (np.abs(frac - 0.5) < window) & (np.repeat(np.asarray(s), np.asarray(v).shape[-1] // np.asarray(s).shape[-1],
                                                        axis=-1) > 0)
 
 
-def check_block(rec, dbg: dict | None, oq: dict, T: int, D: int, layout: int) -> dict:
-    """Compare one GPU record (+ optional fp32 debug scales) against an oracle quantize_block result."""
+def check_block(rec, dbg: dict | None, oq: dict, T: int, D: int, layout: int, rtol: float = None,
+                window: float = None) -> dict:
+    """Compare one GPU record (+ optional fp32 debug scales) against an oracle quantize_block result.
+
+    rtol (scales) and window (codes, binary16 midpoints) default to the contract's 1e-5; a looser value is only
+    for blocks whose scales are ill-conditioned in fp32, with the reason stated where it is used."""
+    rtol = SCALE_RTOL if rtol is None else rtol
+    window = WINDOW if window is None else window
     g = view_record(rec, T, D, layout)
-    stats = dict(elements=T * D, boundary=0, code_flips=0, f16_flips=0)
+    stats = dict(elements=T * D, boundary=0, code_flips=0, f16_flips=0, max_rel=0.0)
     # codes
-    nb = near_boundary(oq["v"], oq["s"])
+    nb = near_boundary(oq["v"], oq["s"], window)
     mism = g["codes"] != oq["codes"]
     bad = mism & ~nb
     assert not bad.any(), f"{int(bad.sum())} code mismatches outside the rounding window, e.g. at " \
@@ -93,8 +101,11 @@ def check_block(rec, dbg: dict | None, oq: dict, T: int, D: int, layout: int) ->
             o = np.asarray(oq[key], dtype=np.float64)
             gv = np.asarray(dbg[key], dtype=np.float64).reshape(o.shape)
             err = np.abs(gv - o)
-            tol = SCALE_RTOL * np.abs(o)
+            tol = rtol * np.abs(o)
             ok = (err <= tol) | ((o == 0) & (err == 0))
+            nzo = o != 0
+            if nzo.any():
+                stats["max_rel"] = max(stats["max_rel"], float(np.max(err[nzo] / np.abs(o[nzo]))))
             assert ok.all(), f"{key}: max rel err {np.max(err / np.maximum(np.abs(o), 1e-300)):.3e}"
     # stored binary16 scales
     for key in ("r", "c", "s", "m"):
@@ -102,7 +113,7 @@ def check_block(rec, dbg: dict | None, oq: dict, T: int, D: int, layout: int) ->
         expect = o.astype(np.float16)
         got = g[key].reshape(o.shape)
         diff = expect.view(np.uint16) != got.view(np.uint16)
-        near = near_f16_midpoint(o)
+        near = near_f16_midpoint(o, max(window, rtol))
         assert not (diff & ~near).any(), f"binary16 {key} differs away from a midpoint at " \
                                          f"{np.argwhere(diff & ~near)[:5].tolist()}"
         stats["f16_flips"] += int(diff.sum())
