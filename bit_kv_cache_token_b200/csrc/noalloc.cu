@@ -7,7 +7,10 @@
 // them this entry point uses a workspace that lives in this library's own
 // device image: a file-scope __device__ array, reserved on every GPU that
 // loads the library and held until the process exits.
+#include <cuda.h>
 #include <cuda_runtime.h>
+
+#include <mutex>
 
 #include "kvarn.h"
 
@@ -18,20 +21,79 @@ constexpr size_t kStaticScratchBytes = (size_t)16 << 20;
 
 __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
 
-// Device address of g_decode_scratch, looked up once per device.  In host
-// code the symbol name is only a host-side stand-in, never a device address.
-void *g_scratch_ptr[64] = {nullptr};
+// In host code g_decode_scratch is only a host-side stand-in, never a device
+// address.  Its device address belongs to one CUDA context (a second context
+// on the same device, or the context created again after cudaDeviceReset,
+// loads the module anew at another address), so the looked-up address is
+// cached per context, keyed by the driver's unique context id.  The cache is
+// shared by all host threads and guarded by a mutex.
+struct ScratchEntry {
+    unsigned long long ctx_id;
+    void *ptr;
+};
+constexpr int kCacheSlots = 64;
+std::mutex g_mu;
+ScratchEntry g_cache[kCacheSlots];
+int g_used = 0, g_next = 0;
 
-int scratch_for_current_device(void **out)
+using PfnCtxGetCurrent = CUresult (*)(CUcontext *);
+using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long *);
+PfnCtxGetCurrent g_get_current = nullptr;
+PfnCtxGetId g_get_id = nullptr;
+bool g_resolved = false;
+
+// Driver entry points, resolved once through the runtime (no link-time
+// dependency on the driver library).  Called with g_mu held.
+void resolve_entry_points()
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return KVARN_ECUDA;
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return KVARN_ECUDA;
-        g_scratch_ptr[dev] = p;
+    if (g_resolved) return;
+    g_resolved = true;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        g_get_current = reinterpret_cast<PfnCtxGetCurrent>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        g_get_id = reinterpret_cast<PfnCtxGetId>(fn);
+}
+
+// Unique id of the calling thread's current context; false when there is
+// none yet or the driver cannot tell.
+bool current_context_id(unsigned long long *id)
+{
+    if (!g_get_current || !g_get_id) return false;
+    CUcontext ctx = nullptr;
+    if (g_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+    return g_get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_decode_scratch in the current context.  The first
+// call in a context looks it up (cudaGetSymbolAddress, which also sets up the
+// device's primary context if none is current) and caches it.
+int scratch_for_current_context(void **out)
+{
+    std::lock_guard<std::mutex> lock(g_mu);
+    resolve_entry_points();
+    unsigned long long id = 0;
+    bool have_id = current_context_id(&id);
+    if (have_id) {
+        for (int i = 0; i < g_used; ++i)
+            if (g_cache[i].ctx_id == id) {
+                *out = g_cache[i].ptr;
+                return KVARN_OK;
+            }
     }
-    *out = g_scratch_ptr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return KVARN_ECUDA;
+    if (!have_id) have_id = current_context_id(&id);  // the lookup may have made the context current
+    if (have_id) {
+        g_cache[g_next] = ScratchEntry{id, p};
+        g_next = (g_next + 1) % kCacheSlots;
+        if (g_used < kCacheSlots) ++g_used;
+    }
+    *out = p;
     return KVARN_OK;
 }
 
@@ -46,7 +108,7 @@ int kvarn_decode_attention_noalloc(const kvarn_config *cfg, const void *q, int n
     if (need == 0) return KVARN_EINVAL;
     if (need > kStaticScratchBytes) return KVARN_EWORKSPACE;
     void *ws = nullptr;
-    const int rc = scratch_for_current_device(&ws);
+    const int rc = scratch_for_current_context(&ws);
     if (rc != KVARN_OK) return rc;
     // The array keeps the previous call's contents: the split tickets at its
     // start must be zero when a decode begins.

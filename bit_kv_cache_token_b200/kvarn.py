@@ -192,9 +192,19 @@ def _need(t, name, dtype=None, shape=None):
 
 
 def _on_device(**tensors):
+    """Every tensor must live on the current CUDA device: the library launches on the current device (its
+    stream, its SM count, and for the no-alloc decode its own copy of the static workspace)."""
+    cur = None
     for name, t in tensors.items():
-        if t is not None and not t.is_cuda:
+        if t is None:
+            continue
+        if not t.is_cuda:
             raise ValueError(f"{name} must be a CUDA tensor")
+        if cur is None:
+            cur = torch.cuda.current_device()
+        if t.device.index != cur:
+            raise ValueError(f"{name} is on cuda:{t.device.index} but the current device is cuda:{cur}; "
+                             f"call inside torch.cuda.device({t.device.index})")
 
 
 def _need_cache(cfg: Config, cache: KVCache):

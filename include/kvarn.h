@@ -157,6 +157,11 @@ KVARN_API size_t kvarn_decode_workspace_bytes(const kvarn_config *cfg, int num_q
  * Bulk quantisation (prefill) of num_tokens tokens per sequence, written as
  * tokens first_block*T .. first_block*T + num_tokens - 1:
  *   k, v  [num_seqs][num_kv_heads][num_tokens][D] in cfg->dtype.
+ * Source: the abstract (Hadamard rotation, dual-scaling variance
+ * normalisation across the token and channel axes of K and V, 2-bit
+ * codes) and the rndamp.com article, "How It Works", items 1 (Hadamard
+ * transform in the channel dimension) and 2 (iterative balancing of rows
+ * and columns until the variance is close to uniform).
  * Full blocks go through rotation -> normalisation -> 2-bit packing into
  * record slots first_block, first_block+1, ...; the last num_tokens % T
  * tokens are copied, unrotated, into the tail; n_tokens[s] is set to
@@ -173,6 +178,9 @@ KVARN_API int kvarn_quantize_blocks(const kvarn_config *cfg, const void *k, cons
                           float *debug_k, float *debug_v, void *stream);
 
 /*
+ * Source: the abstract (the cache grows with every decoded token in
+ * long-horizon decoding) and the rndamp.com article, "How It Works" (each
+ * full block is rotated, normalised and coded as in kvarn_quantize_blocks).
  * Append one token per sequence (k, v: [num_seqs][num_kv_heads][D]) at
  * position n_tokens[s].  The token goes into tail slot n % T; when that fills
  * the tail, the tail is quantised into record n / T in the same launch.
@@ -183,6 +191,11 @@ KVARN_API int kvarn_append_token(const kvarn_config *cfg, const void *k, const v
                        const kvarn_cache *cache, void *stream);
 
 /*
+ * Source: the abstract (decode attention over the 2-bit cache, which is
+ * what bounds long-horizon decoding) and the rndamp.com article, "Numbers"
+ * (the second scale is fused into the dequantisation inside the attention
+ * kernel); the query is rotated like the keys ("How It Works", item 1: the
+ * rotation is orthogonal, so q . k is unchanged).
  * Single-token decode attention over the whole cache:
  *   q    [num_seqs][num_q_heads][D] in cfg->dtype, unrotated;
  *   out  [num_seqs][num_q_heads][D] fp32, unrotated;
@@ -259,6 +272,9 @@ KVARN_API int kvarn_token_errors(const kvarn_config *cfg, const void *k, const v
                                  void *stream);
 
 /*
+ * Source: the rndamp.com article, "Numbers" (each value is rebuilt from its
+ * code with both scales, r_t c_d (s code + m)) and "How It Works", item 1
+ * (the rotation is its own inverse once normalised).
  * Dequantise records first_block .. first_block+num_blocks-1 of every
  * (sequence, kv head) into fp32 k_out / v_out
  * [num_seqs][num_kv_heads][num_blocks*T][D]; rotated != 0 keeps the rotated
@@ -279,8 +295,11 @@ KVARN_API int kvarn_dequantize(const kvarn_config *cfg, const kvarn_cache *cache
  * on every GPU that loads it, until the process exits; a call whose
  * kvarn_decode_workspace_bytes(cfg, num_q_heads) exceeds 16 MiB returns
  * KVARN_EWORKSPACE.  Nothing is allocated or freed.
- * The first call on a device looks up the array's device address (with that
- * device current); make that first call before any stream capture.  Every
+ * The first call in a CUDA context looks up the array's device address in
+ * that context (with it current) and caches it for that context; make that
+ * first call before any stream capture.  The cache is keyed by the driver's
+ * context id, so other contexts on the same device, and a context created
+ * again after cudaDeviceReset, get their own lookup.  Every
  * call clears the array's combine tickets on `stream` and then uses the
  * array, so calls whose work overlaps on the GPU (any two streams, any two
  * threads) race with each other: order them.  Arguments and results are as

@@ -28,7 +28,8 @@ def test_noalloc_decode_matches_workspace_decode_twice_in_a_row():
         kvarn.decode_attention_noalloc(cfg, q, cache, L, out)
         torch.cuda.synchronize()
         assert int(cache.status.item()) == 0
-        np.testing.assert_allclose(out.cpu().numpy(), ref.cpu().numpy(), rtol=0, atol=2e-3)
+        # the same kernel on the same inputs, and decode is deterministic: bit-identical
+        assert torch.equal(out, ref)
 
 
 def test_noalloc_rejects_a_workspace_beyond_the_static_size():
