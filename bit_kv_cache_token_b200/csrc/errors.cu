@@ -24,7 +24,7 @@ token_errors_kernel(ErrorArgs a)
     using R = Record<D>;
     constexpr int W = D / 32;
     constexpr int NG = D / kGroup;
-    __shared__ QuantSmem<D> sm;
+    QuantSmem<D> &sm = quant_smem<D>();
     __shared__ float red[3][W][kBlockTokens];
     const int j = threadIdx.x >> 5, l = threadIdx.x & 31;
     const int nb = a.num_blocks;
@@ -45,7 +45,7 @@ token_errors_kernel(ErrorArgs a)
     const __half *ch16 = reinterpret_cast<const __half *>(rec + R::kCOff);
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        const int t = l + 32 * r;
+        const int t = qtok(l) + 32 * r;
         const float rt = __half2float(rh16[t]);
         const float s = __half2float(sh16[t * NG + j]), m = __half2float(mh16[t * NG + j]);
         float xx = 0.f, yy = 0.f, xy = 0.f;
@@ -92,7 +92,11 @@ template <int D, int HB, typename Tin>
 static cudaError_t launch_err(const ErrorArgs &a, int units, cudaStream_t st)
 {
     dim3 grid((unsigned)(units * a.num_blocks), 2);
-    token_errors_kernel<D, HB, Tin><<<grid, D, 0, st>>>(a);
+    constexpr int kSmem = (int)sizeof(QuantSmem<D>);
+    const cudaError_t e =
+        cudaFuncSetAttribute(token_errors_kernel<D, HB, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
+    token_errors_kernel<D, HB, Tin><<<grid, D, kSmem, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -4,17 +4,34 @@
 
 namespace kvarn {
 
+// Load a block and quantise it: bf16 blocks are rotated on the tensor cores,
+// fp32 blocks on the CUDA cores.
+template <int D, int HB, typename Tin, bool COHERENT>
+__device__ __forceinline__ void load_quantize(const Tin *src, QuantSmem<D> &sm, int tensor, int sweeps,
+                                              unsigned char *rec, float *dbg, int32_t *status)
+{
+    float2 X[4][16];
+    if constexpr (sizeof(Tin) == 2) {
+        load_rotate_tc<D, HB>(src, X, sm);  // reads through L2: coherent either way
+        if (tensor) quantize_block<D, HB, 1, true>(X, sm, sweeps, rec, dbg, status);
+        else quantize_block<D, HB, 0, true>(X, sm, sweeps, rec, dbg, status);
+    } else {
+        load_block<D, Tin, COHERENT>(src, X);
+        if (tensor) quantize_block<D, HB, 1>(X, sm, sweeps, rec, dbg, status);
+        else quantize_block<D, HB, 0>(X, sm, sweeps, rec, dbg, status);
+    }
+}
+
 // One CTA per (sequence, kv head, block) and per tensor (blockIdx.y: 0 = K,
 // 1 = V).  Block index nb (one past the full blocks) copies the ragged tail.
 // 12 warps per SM: the register cap (168) spills a few words of the 128-float
 // block a thread holds, yet the extra warps hide more of the dependent
-// arithmetic's latency than the spills cost (705.7 -> 673.0 us for 16 x 8 x
-// 8192 bf16 tokens of K and V at D = 128).
+// arithmetic's latency than the spills cost.
 template <int D, int HB, typename Tin>
 __global__ void __launch_bounds__(D, 384 / D)
 quantize_blocks_kernel(QuantArgs a)
 {
-    __shared__ QuantSmem<D> sm;
+    QuantSmem<D> &sm = quant_smem<D>();
     const int nb = a.num_tokens / kBlockTokens;
     const int rem = a.num_tokens % kBlockTokens;
     const int nbx = nb + (rem > 0 ? 1 : 0);
@@ -32,15 +49,12 @@ quantize_blocks_kernel(QuantArgs a)
         copy_elems(tail, src, rem * D, threadIdx.x, D);
         return;
     }
-    float2 X[4][16];
-    load_block<D>(src, X);
     const size_t slot = (size_t)sh * a.max_blocks + a.first_block + b;
     unsigned char *rec = static_cast<unsigned char *>(tensor ? a.v_records : a.k_records) +
                          slot * Record<D>::kBytes;
     float *dbg = tensor ? a.debug_v : a.debug_k;
     if (dbg) dbg += ((size_t)sh * nb + b) * (kBlockTokens + D + 2 * kBlockTokens * (D / kGroup));
-    if (tensor) quantize_block<D, HB, 1>(X, sm, a.sweeps, rec, dbg, a.status);
-    else quantize_block<D, HB, 0>(X, sm, a.sweeps, rec, dbg, a.status);
+    load_quantize<D, HB, Tin, false>(src, sm, tensor, a.sweeps, rec, dbg, a.status);
 }
 
 // One CTA per (sequence, kv head) and per tensor.  The token goes into tail
@@ -51,7 +65,7 @@ template <int D, int HB, typename Tin>
 __global__ void __launch_bounds__(D, 2)
 append_kernel(AppendArgs a)
 {
-    __shared__ QuantSmem<D> sm;
+    QuantSmem<D> &sm = quant_smem<D>();
     __shared__ int s_n;
     const int sh = blockIdx.x;  // s * Hkv + h
     const int s = sh / a.num_kv_heads;
@@ -69,12 +83,10 @@ append_kernel(AppendArgs a)
         copy_elems(tail + (size_t)pos * D, tok, D, threadIdx.x, D);
         if (fills) {
             __syncthreads();  // the new row is visible to the whole CTA
-            float2 X[4][16];
-            load_block<D, Tin, true>(tail, X);  // row pos was just written by this CTA
             unsigned char *rec = static_cast<unsigned char *>(tensor ? a.v_records : a.k_records) +
                                  ((size_t)sh * a.max_blocks + blk) * Record<D>::kBytes;
-            if (tensor) quantize_block<D, HB, 1>(X, sm, a.sweeps, rec, nullptr, a.status);
-            else quantize_block<D, HB, 0>(X, sm, a.sweeps, rec, nullptr, a.status);
+            // row pos was just written by this CTA: read the tail through L2
+            load_quantize<D, HB, Tin, true>(tail, sm, tensor, a.sweeps, rec, nullptr, a.status);
         }
     } else if (threadIdx.x == 0 && tensor == 0 && (sh % a.num_kv_heads) == 0) {
         status_or(a.status, KVARN_STATUS_CAPACITY);
@@ -98,7 +110,13 @@ static cudaError_t launch_quant(const QuantArgs &a, int S, int Hkv, cudaStream_t
     const int nbx = nb + (a.num_tokens % kBlockTokens ? 1 : 0);
     if (nbx == 0) return cudaSuccess;
     dim3 grid((unsigned)(S * Hkv * nbx), 2);
-    quantize_blocks_kernel<D, HB, Tin><<<grid, D, 0, st>>>(a);
+    constexpr int kSmem = (int)sizeof(QuantSmem<D>);
+    const cudaError_t e =
+        cudaFuncSetAttribute(quantize_blocks_kernel<D, HB, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
+    // the largest shared-memory carveout, so that three CTAs fit on an SM
+    cudaFuncSetAttribute(quantize_blocks_kernel<D, HB, Tin>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    quantize_blocks_kernel<D, HB, Tin><<<grid, D, kSmem, st>>>(a);
     return cudaGetLastError();
 }
 
@@ -106,7 +124,13 @@ template <int D, int HB, typename Tin>
 static cudaError_t launch_append(const AppendArgs &a, int S, int Hkv, cudaStream_t st)
 {
     dim3 grid((unsigned)(S * Hkv), 2);
-    append_kernel<D, HB, Tin><<<grid, D, 0, st>>>(a);
+    constexpr int kSmem = (int)sizeof(QuantSmem<D>);
+    const cudaError_t e =
+        cudaFuncSetAttribute(append_kernel<D, HB, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
+    // the largest shared-memory carveout, so that three CTAs fit on an SM
+    cudaFuncSetAttribute(append_kernel<D, HB, Tin>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    append_kernel<D, HB, Tin><<<grid, D, kSmem, st>>>(a);
     return cudaGetLastError();
 }
 

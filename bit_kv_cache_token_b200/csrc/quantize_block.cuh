@@ -18,19 +18,38 @@
 //   4. store codes, binary16 (s, m), r and c in one block record.
 //
 // Thread layout (D threads = D/32 warps; warp j owns channel group j):
-// lane l holds tokens l, l+32, l+64, l+96 and channels 32j .. 32j+31 of each,
-// as 16 float2 per token.  So a quantisation group sits entirely in one
-// thread, the 32-point Hadamard butterflies are in registers, a larger
-// Hadamard block adds one exchange across warps through shared memory, the
-// per-token (row) sums cross warps through shared memory and the
+// lane l holds tokens qtok(l) + 32r (r = 0..3) and channels 32j .. 32j+31 of
+// each, as 16 float2 per token.  So a quantisation group sits entirely in one
+// thread, the per-token (row) sums cross warps through shared memory and the
 // per-channel (column) sums cross the 32 lanes through a swizzled
-// shared-memory transpose.  Arithmetic is fp32; packed f32x2 operations
-// (sm_100) halve the issue count of the elementwise work.
+// shared-memory transpose.
+// Rotation.  bf16 blocks are rotated on the tensor cores: the Hadamard matrix
+// is +-1, exact in bf16, and the products accumulate in fp32, so X H is a
+// plain dense contraction (mma.sync m16n8k16).  Warp j computes its group's
+// 32 outputs from the HB inputs of its Hadamard block, all 128 tokens, with
+// A fragments read by ldmatrix from the block staged in shared memory.  fp32
+// blocks take the CUDA-core path: 32-point butterflies in registers and one
+// exchange across warps per further channel bit.  Arithmetic is fp32; packed
+// f32x2 operations (sm_100) halve the issue count of the elementwise work.
 #pragma once
 
 #include "kvarn_common.cuh"
 
 namespace kvarn {
+
+// Lane l's first token: lanes 4g + tig hold tokens 8 tig + g (+ 32 r), the
+// order in which the tensor-core rotation leaves them.
+__host__ __device__ constexpr int qtok(int l) { return 8 * (l & 3) + (l >> 2); }
+
+// Shared-memory stage of the tensor-core rotation: the bf16 block, rows padded
+// by 16 bytes so that the eight row addresses of an ldmatrix hit distinct
+// banks, and one 32-token x 32-channel fp32 transpose buffer per warp.
+template <int D>
+struct TcStage {
+    static constexpr int kRowBytes = 2 * D + 16;
+    unsigned char rows[kBlockTokens * kRowBytes];
+    float4 xbuf[D / 32][32][8];
+};
 
 template <int D>
 struct QuantSmem {
@@ -39,6 +58,7 @@ struct QuantSmem {
         float4 xch[W][2][8][32];               // Hadamard exchange [warp][token pair][chunk][lane]
         float4 col[W][32][16];                 // column-sum transpose [warp][lane][chunk]
         unsigned char rec[Record<D>::kBytes];  // record staging
+        TcStage<D> tc;                         // tensor-core rotation (bf16 blocks)
     } u;
     float part[2][W][kBlockTokens];            // per-token partial row sums: [0] of z, [1] of (z - mean)^2
     float ubuf[D];                             // 1 / c broadcast
@@ -46,6 +66,15 @@ struct QuantSmem {
     float2 gpart[W];                           // per-warp (sum of log2 c, count) of nonzero-variance channels
     float ymax[W][kBlockTokens];               // per-(group, token) largest |Y| (token gauge)
 };
+
+// The block quantiser's shared memory lives in the dynamic segment (it exceeds
+// the 48 KB static limit at D = 128); launches pass sizeof(QuantSmem<D>).
+template <int D>
+__device__ __forceinline__ QuantSmem<D> &quant_smem()
+{
+    extern __shared__ __align__(16) unsigned char quant_smem_raw[];
+    return *reinterpret_cast<QuantSmem<D> *>(quant_smem_raw);
+}
 
 // A variance at most this fraction of the mean square counts as zero.  In
 // fp32, values that are all equal leave a residual of order 2^-48 of their
@@ -99,7 +128,7 @@ __device__ __forceinline__ void load_block(const Tin *rows, float2 (&X)[4][16])
     const int j = threadIdx.x >> 5, l = threadIdx.x & 31;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        const Tin *p = rows + (size_t)(l + 32 * r) * D + 32 * j;
+        const Tin *p = rows + (size_t)(qtok(l) + 32 * r) * D + 32 * j;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             float v[8];
@@ -157,11 +186,198 @@ __device__ __forceinline__ void rotate_block(float2 (&X)[4][16], QuantSmem<D> &s
 
 }
 
+// ---- tensor-core rotation of a bf16 block --------------------------------
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The same with a zero accumulator in (the first k-tile of a chain).
+__device__ __forceinline__ void mma_bf16_16816_z(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};\n"
+        : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&a)[4], const void *p)
+{
+    const uint32_t addr = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                 : "r"(addr));
+}
+
+// Copy the 128 x D bf16 rows into the padded stage with asynchronous 16-byte
+// copies (cp.async.cg: no register round trip, every copy of the thread in
+// flight at once, read through L2 -- which also sees the append path's tail
+// that this kernel wrote before a CTA barrier).  The caller waits and syncs.
+template <int D>
+__device__ __forceinline__ void stage_rows(const __nv_bfloat16 *rows, TcStage<D> &st)
+{
+    constexpr int CH = D / 8;  // 16-byte chunks per row
+    constexpr int N = kBlockTokens * CH / D;  // copies per thread (D threads): 16 at every D
+    static_assert(kBlockTokens * CH % D == 0, "stage split");
+#pragma unroll
+    for (int it = 0; it < N; ++it) {
+        const int i = threadIdx.x + it * D;
+        const int row = i / CH, ch = i % CH;
+        const void *src = rows + (size_t)row * D + 8 * ch;
+        const uint32_t dst = static_cast<uint32_t>(
+            __cvta_generic_to_shared(st.rows + row * TcStage<D>::kRowBytes + 16 * ch));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+    }
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+}
+
+// Physical float4 slot of logical slot q in row `row` of a transpose buffer:
+// the eight lanes of one 16-byte read phase then hit distinct banks.
+__device__ __forceinline__ int xswz(int row, int q) { return q ^ ((((row >> 3) << 1) | (row & 1)) & 7); }
+
+// One warp's share of X H for a bf16 block: the 32 rotated channels of group j
+// (unnormalised: the stored r takes the 1/sqrt(HB)), all 128 tokens, into X
+// in the thread layout.  HB in {0, 32, 64, 128}.
+//
+// Output channel 32j + 8 nu + n of n-tile nu is column n of the MMA; input
+// channel 16 kappa + k of the warp's Hadamard block is row k of k-tile kappa.
+// With i = 16 kappa + k and o = 32 JP + 8 nu + n (both within the block,
+// JP = j mod (HB / 32)),
+//   (-1)^popcount(i & o) = (-1)^popcount(k & (8 (nu & 1) + n))
+//                        * (-1)^popcount(kappa & (nu >> 1))
+//                        * (-1)^popcount(kappa & 2 JP),
+// a per-lane base fragment (two of them, by nu & 1), a sign fixed at compile
+// time, and a sign set by the warp.  The last is either 1 for every kappa
+// (JP = 0) or, once the k-tiles are visited in a warp-chosen order, kappa's
+// bit 1 (JP = 2: bits 1 and 2 of kappa swapped; JP = 3: bit 1 replaced by
+// bit 1 xor bit 2), so one code path serves every warp: the k-tiles with bit 1
+// set use base registers whose signs the warp swapped once.
+// m-tile mu of round rho holds tokens 32 rho + 16 mu + (0..15); the C
+// fragments leave lane (g, tig) tokens g + {0, 8, 16, 24} x channels
+// 8 nu + 2 tig + {0, 1}, and a transpose through the warp's buffer gives lane
+// 4g + tig the token 8 tig + g = qtok(lane) with all 32 channels.
+template <int D, int HB>
+__device__ __forceinline__ void rotate_warp_tc(float2 (&X)[4][16], TcStage<D> &st)
+{
+    const int j = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, tig = lane & 3;
+    constexpr uint32_t kOne = 0x3F80u, kMinus = 0xBF80u;  // bf16 +1, -1
+    // base B fragments: b0 holds rows k = 2 tig + {0, 1}, b1 rows k = 2 tig + 8 + {0, 1}, column n = g
+    uint32_t bp[2][2], bn[2][2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            uint32_t reg = 0u;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int k = 2 * tig + 8 * half + e;
+                uint32_t v;
+                if constexpr (HB == 0) v = (k == 8 * h + g) ? kOne : 0u;  // identity
+                else v = (__popc(k & (8 * h + g)) & 1) ? kMinus : kOne;
+                reg |= v << (16 * e);
+            }
+            bp[h][half] = reg;
+            bn[h][half] = reg ^ 0x80008000u;
+        }
+    constexpr int NKT = HB == 0 ? 2 : HB / 16;  // k-tiles feeding this warp
+    const int jp = HB >= 64 ? j % (HB / 32) : 0;
+    // the warp's sign on k-tiles with bit 1 set: swap the bases' signs once
+    const bool flip = jp != 0;
+    uint32_t sp[2][2], sn[2][2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            sp[h][half] = flip ? bn[h][half] : bp[h][half];
+            sn[h][half] = flip ? bp[h][half] : bn[h][half];
+        }
+    // byte offset of each k-tile in a staged row, in the warp's visiting order
+    const int kt0 = HB == 0 ? 2 * j : (32 * j / (HB == 0 ? 32 : HB)) * (HB / 16);
+    int koff[NKT];
+#pragma unroll
+    for (int kap = 0; kap < NKT; ++kap) {
+        int kk = kap;
+        if (HB == 128 && jp == 2) kk = (kap & 1) | ((kap & 2) << 1) | ((kap & 4) >> 1);
+        if (HB == 128 && jp == 3) kk = kap ^ ((kap & 4) >> 1);
+        koff[kap] = 32 * (kt0 + kk);
+    }
+    float4(&xb)[32][8] = st.xbuf[j];
+#pragma unroll
+    for (int rho = 0; rho < 4; ++rho) {  // unrolled: X[rho] must stay in registers
+#pragma unroll
+        for (int mu = 0; mu < 2; ++mu) {
+            float acc[4][4];
+            const int arow = 32 * rho + 16 * mu + (lane & 7) + 8 * ((lane >> 3) & 1);
+            const unsigned char *abase = st.rows + arow * TcStage<D>::kRowBytes + 16 * (lane >> 4);
+#pragma unroll
+            for (int kap = 0; kap < NKT; ++kap) {
+                uint32_t a[4];
+                ldmatrix_x4(a, abase + koff[kap]);
+#pragma unroll
+                for (int nu = 0; nu < 4; ++nu) {
+                    if constexpr (HB == 0) {
+                        // identity: k-tile 2j + (nu >> 1) alone feeds n-tile nu
+                        if (kap != (nu >> 1)) continue;
+                        mma_bf16_16816_z(acc[nu], a, bp[nu & 1][0], bp[nu & 1][1]);
+                    } else {
+                        const bool neg = __popc(kap & (nu >> 1)) & 1;  // compile-time
+                        const uint32_t b0 = (kap & 2) == 0 ? (neg ? bn[nu & 1][0] : bp[nu & 1][0])
+                                                           : (neg ? sn[nu & 1][0] : sp[nu & 1][0]);
+                        const uint32_t b1 = (kap & 2) == 0 ? (neg ? bn[nu & 1][1] : bp[nu & 1][1])
+                                                           : (neg ? sn[nu & 1][1] : sp[nu & 1][1]);
+                        if (kap == 0) mma_bf16_16816_z(acc[nu], a, b0, b1);
+                        else mma_bf16_16816(acc[nu], a, b0, b1);
+                    }
+                }
+            }
+            // C fragments -> transpose buffer: rows 16 mu + g (c0, c1) and 16 mu + g + 8 (c2, c3)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int row = 16 * mu + g + 8 * hh;
+#pragma unroll
+                for (int nu = 0; nu < 4; ++nu) {
+                    const int q = 2 * nu + (tig >> 1);  // channel 8 nu + 2 tig sits in float4 q, half tig & 1
+                    float2 *dst = reinterpret_cast<float2 *>(&xb[row][xswz(row, q)]) + (tig & 1);
+                    *dst = f2(acc[nu][2 * hh], acc[nu][2 * hh + 1]);
+                }
+            }
+        }
+        __syncwarp();
+        const int row = qtok(lane);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float4 v = xb[row][xswz(row, q)];
+            X[rho][2 * q] = f2(v.x, v.y);
+            X[rho][2 * q + 1] = f2(v.z, v.w);
+        }
+        __syncwarp();
+    }
+}
+
+// Load and rotate a bf16 block on the tensor cores (all D threads call this).
+template <int D, int HB>
+__device__ __forceinline__ void load_rotate_tc(const __nv_bfloat16 *rows, float2 (&X)[4][16], QuantSmem<D> &sm)
+{
+    stage_rows<D>(rows, sm.u.tc);
+    __syncthreads();
+    rotate_warp_tc<D, HB>(X, sm.u.tc);
+    __syncthreads();  // the stage is free for the union's next use
+}
+
 // Quantise the block held in X (destroyed) into rec_out (global, 16-byte
 // aligned, Record<D>::kBytes); TENSOR 0 = K code order, 1 = V code order.
 // dbg: NULL or fp32 [T + D + 2*T*D/32] unrounded r, c, s, m (as stored, token
 // gauge included).  All D threads of the CTA must call this.
-template <int D, int HB, int TENSOR>
+// PREROT: X already holds the rotation, unnormalised (tensor-core path); the
+// 1/sqrt(HB) then goes into the stored r (Y, c, s and m do not depend on it).
+template <int D, int HB, int TENSOR, bool PREROT = false>
 __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
                                unsigned char *__restrict__ rec_out, float *__restrict__ dbg,
                                int32_t *status)
@@ -169,9 +385,15 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
     constexpr int W = D / 32;
     using R = Record<D>;
     const int j = threadIdx.x >> 5, l = threadIdx.x & 31;
+    const int t0 = qtok(l);  // this lane's tokens: t0 + 32 r
+    // 1/sqrt(HB) of a rotation left unnormalised
+    constexpr float kRNorm = !PREROT || HB == 0 ? 1.f : HB == 32 ? 0.17677669529663688f
+                                                       : HB == 64 ? 0.125f : 0.08838834764831845f;
+    // a token scale of 1 (no sweeps, zero-variance row) in the frame of X
+    constexpr float kRUnit = 1.f / kRNorm;
 
     // ---- 1. Hadamard rotation along the channels --------------------------
-    rotate_block<D, HB>(X, sm);
+    if constexpr (!PREROT) rotate_block<D, HB>(X, sm);
 
     // ---- 2. dual-axis variance normalisation ------------------------------
     // Rows: two passes (mean, then mean square deviation) over the D channels,
@@ -180,26 +402,31 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
     // whose partials cross the lanes through a shared-memory transpose.  Then
     // the gauge: g = geometric mean of the nonzero-variance channel scales,
     // c <- c / g (1 for a zero-variance column), r <- r g at the end.
-    float2 u[16];  // 1 / c for this thread's 32 channels
-#pragma unroll
-    for (int k = 0; k < 16; ++k) u[k] = f2(1.f, 1.f);
-    float w[4] = {1.f, 1.f, 1.f, 1.f};    // 1 / r for this thread's 4 tokens
-    float rt[4] = {1.f, 1.f, 1.f, 1.f};   // r for this thread's 4 tokens (0 marks zero variance)
+    // 1 / c of the warp's 32 channels lives in sm.ubuf (the same for every
+    // lane of the warp: broadcast reads, channel-outer loops), not in registers
+    sm.ubuf[32 * j + l] = 1.f;
+    __syncwarp();
+    const float2 *u2 = reinterpret_cast<const float2 *>(&sm.ubuf[32 * j]);
+    float w[4] = {kRNorm, kRNorm, kRNorm, kRNorm};  // 1 / r for this thread's 4 tokens
+    float rt[4] = {0.f, 0.f, 0.f, 0.f};   // r for this thread's 4 tokens (0: scale 1, kRUnit in X's frame)
     float cd = 1.f;                       // c of channel 32j + l (lane-owned, gauged)
     float g = 1.f;                        // gauge factor of the last column step
 
     for (int sw = 0; sw < sweeps; ++sw) {
         // row step, pass 1: mean over the D channels of z = X u
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            float2 s1 = f2(0.f, 0.f), s1b = f2(0.f, 0.f);
+        {
+            float2 s1[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
             for (int k = 0; k < 16; k += 2) {
-                s1 = __ffma2_rn(X[r][k], u[k], s1);
-                s1b = __ffma2_rn(X[r][k + 1], u[k + 1], s1b);
+                const float4 u4 = reinterpret_cast<const float4 *>(u2)[k >> 1];  // one broadcast read, two pairs
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    s1[r] = __ffma2_rn(X[r][k], f2(u4.x, u4.y), s1[r]);
+                    s1[r] = __ffma2_rn(X[r][k + 1], f2(u4.z, u4.w), s1[r]);
+                }
             }
-            s1 = __fadd2_rn(s1, s1b);
-            sm.part[0][j][l + 32 * r] = s1.x + s1.y;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) sm.part[0][j][t0 + 32 * r] = s1[r].x + s1[r].y;
         }
         __syncthreads();
         float mean[4];
@@ -207,38 +434,40 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
         for (int r = 0; r < 4; ++r) {
             float S1 = 0.f;
 #pragma unroll
-            for (int jj = 0; jj < W; ++jj) S1 += sm.part[0][jj][l + 32 * r];
+            for (int jj = 0; jj < W; ++jj) S1 += sm.part[0][jj][t0 + 32 * r];
             mean[r] = S1 * (1.f / D);
         }
         // row step, pass 2: mean square deviation from that mean
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const float2 nm = f2(-mean[r], -mean[r]);
-            float2 s2 = f2(0.f, 0.f), s2b = f2(0.f, 0.f);
+        {
+            float2 s2[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
             for (int k = 0; k < 16; k += 2) {
-                const float2 e = __ffma2_rn(X[r][k], u[k], nm);
-                const float2 eb = __ffma2_rn(X[r][k + 1], u[k + 1], nm);
-                s2 = __ffma2_rn(e, e, s2);
-                s2b = __ffma2_rn(eb, eb, s2b);
+                const float4 u4 = reinterpret_cast<const float4 *>(u2)[k >> 1];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const float2 e = __ffma2_rn(X[r][k], f2(u4.x, u4.y), f2(-mean[r], -mean[r]));
+                    const float2 e1 = __ffma2_rn(X[r][k + 1], f2(u4.z, u4.w), f2(-mean[r], -mean[r]));
+                    s2[r] = __ffma2_rn(e, e, s2[r]);
+                    s2[r] = __ffma2_rn(e1, e1, s2[r]);
+                }
             }
-            s2 = __fadd2_rn(s2, s2b);
-            sm.part[1][j][l + 32 * r] = s2.x + s2.y;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) sm.part[1][j][t0 + 32 * r] = s2[r].x + s2[r].y;
         }
         __syncthreads();
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             float S2 = 0.f;
 #pragma unroll
-            for (int jj = 0; jj < W; ++jj) S2 += sm.part[1][jj][l + 32 * r];
+            for (int jj = 0; jj < W; ++jj) S2 += sm.part[1][jj][t0 + 32 * r];
             const float var = S2 * (1.f / D);
             const bool nz = var > kZeroVarRel * fmaf(mean[r], mean[r], var);
             const float is = rsqrtf(var);
-            w[r] = nz ? is : 1.f;         // 1 / r_t
+            w[r] = nz ? is : kRNorm;      // 1 / r_t
             rt[r] = nz ? var * is : 0.f;  // r_t = sqrt(var); 0 marks a zero-variance row (scale 1)
         }
         // column step: c_d = std over the 128 tokens of z = X / r, on values
-        // shifted by token 0's z (lane 0, r = 0) for precision
+        // shifted by token 0's z (lane 0, r = 0: qtok(0) = 0) for precision
         if (l == 0) {
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -253,8 +482,8 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const int k = 8 * half + kk;
-                const float2 kv = reinterpret_cast<const float2 *>(&sm.kbuf[32 * j])[k];
-                const float2 nk = f2(-kv.x, -kv.y);
+                const float4 kv4 = reinterpret_cast<const float4 *>(&sm.kbuf[32 * j])[k >> 1];
+                const float2 nk = (k & 1) ? f2(-kv4.z, -kv4.w) : f2(-kv4.x, -kv4.y);
                 float2 c1 = f2(0.f, 0.f), c2 = f2(0.f, 0.f);
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
@@ -301,18 +530,12 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
             cd = znz ? cd / g : 1.f;
             sm.ubuf[32 * j + l] = 1.f / cd;
             __syncwarp();
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float4 v = reinterpret_cast<const float4 *>(&sm.ubuf[32 * j])[q];
-                u[2 * q] = f2(v.x, v.y);
-                u[2 * q + 1] = f2(v.z, v.w);
-            }
         }
     }
     // last gauge on the token scales: r <- r g (a zero-variance row keeps 1)
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        rt[r] = rt[r] > 0.f ? rt[r] * g : 1.f;
+        rt[r] = rt[r] > 0.f ? rt[r] * g : kRUnit;
         w[r] = 1.f / rt[r];
     }
     __syncthreads();  // every warp is done with the shared transposes
@@ -321,21 +544,30 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
     // Codes go to the record in the fragment order the decode kernel reads
     // (see kvarn.h).  K: the 4 codes of channels 8x + 2*tig + half (x = 0..3)
     // of one token fill one byte.  V: the codes of one channel for this
-    // thread's 4 tokens (l + 32r) fill one byte.
+    // thread's 4 tokens (qtok(l) + 32r) fill one byte.
     unsigned char *rec = sm.u.rec;
     // Codes are read from the low mantissa bits of lev = 1.5*2^23 + code, whose
     // bit pattern is 0x4B400000 + code: multiply-adding the raw patterns with the
     // code weights and subtracting the pattern's share once packs them.
     uint32_t vacc[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // V: channel i in byte i%4 of vacc[i/4]
+    // Z = X u = Y r_t, in place
+#pragma unroll
+    for (int k = 0; k < 16; k += 2) {
+        const float4 u4 = reinterpret_cast<const float4 *>(u2)[k >> 1];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            X[r][k] = __fmul2_rn(X[r][k], f2(u4.x, u4.y));
+            X[r][k + 1] = __fmul2_rn(X[r][k + 1], f2(u4.z, u4.w));
+        }
+    }
     float gs[4], gm[4];  // this group's s and m in Y units, before the token gauge
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        const int t = l + 32 * r;
-        float2 z[16];
+        const int t = t0 + 32 * r;
+        float2 (&z)[16] = X[r];
         float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-            z[k] = __fmul2_rn(X[r][k], u[k]);
             mn = min3(mn, z[k].x, z[k].y);
             mx = max3(mx, z[k].x, z[k].y);
         }
@@ -384,7 +616,7 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
         for (int q = 0; q < 8; ++q) vacc[q] -= kBias;
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-            rec[v_code_bit(l, 32 * j + i) / 8] = (unsigned char)(vacc[i >> 2] >> (8 * (i & 3)));
+            rec[v_code_bit(t0, 32 * j + i) / 8] = (unsigned char)(vacc[i >> 2] >> (8 * (i & 3)));
     }
     __syncthreads();  // every group's largest |Y| is in
     // Token gauge: r_t times the token's (s, m) is what dequantises; when the
@@ -393,7 +625,7 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
     // products unchanged), which keeps s and m inside binary16.
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        const int t = l + 32 * r;
+        const int t = t0 + 32 * r;
         float ym = 0.f;
 #pragma unroll
         for (int jj = 0; jj < W; ++jj) ym = fmaxf(ym, sm.ymax[jj][t]);
@@ -409,7 +641,7 @@ __device__ void quantize_block(float2 (&X)[4][16], QuantSmem<D> &sm, int sweeps,
             status_or(status, KVARN_STATUS_NONFINITE);
         reinterpret_cast<__half *>(rec + R::kSOff)[t * (D / 32) + j] = hs;
         reinterpret_cast<__half *>(rec + R::kMOff)[t * (D / 32) + j] = hm;
-        const float rr = rt[r] * tg;
+        const float rr = rt[r] * tg * kRNorm;
         if (j == 0) {
             const __half hr = __float2half_rn(rr);
             if (__hisinf(hr) || __hisnan(hr)) status_or(status, KVARN_STATUS_NONFINITE);
