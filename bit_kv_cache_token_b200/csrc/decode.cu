@@ -92,9 +92,11 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p)
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// A pure register operation: not volatile, so that independent MMA chains
+// may be interleaved by the compiler.
 __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
 {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};\n"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
@@ -235,25 +237,49 @@ __device__ __forceinline__ bool mbar_wait(unsigned long long *bar, uint32_t pari
 }
 
 // Normalised Walsh-Hadamard transform (block hb, 0 = none) of nvec rows of
-// length D in shared memory, by one warp.
+// length D in shared memory, by one warp.  Lane l holds channels l + 32i of a
+// row: channel bits 0-4 pair lanes (shuffles), bits 5 and 6 pair the lane's
+// own values.
 template <int D>
 __device__ void warp_fwht(float *x, int nvec, int hb)
 {
+    constexpr int NV = D / 32;
     const int lane = threadIdx.x & 31;
     if (hb == 0) return;
-    for (int h = 1; h < hb; h <<= 1) {
-        for (int idx = lane; idx < nvec * D / 2; idx += 32) {
-            const int v = idx / (D / 2), p = idx % (D / 2);
-            const int lo = (p / h) * 2 * h + (p % h);
-            float *row = x + v * D;
-            const float a = row[lo], b = row[lo + h];
-            row[lo] = a + b;
-            row[lo + h] = a - b;
-        }
-        __syncwarp();
-    }
     const float nrm = rsqrtf((float)hb);
-    for (int idx = lane; idx < nvec * D; idx += 32) x[idx] *= nrm;
+    for (int v = 0; v < nvec; ++v) {
+        float *row = x + v * D;
+        float r[NV];
+#pragma unroll
+        for (int i = 0; i < NV; ++i) r[i] = row[lane + 32 * i];
+#pragma unroll
+        for (int bit = 1; bit < 32; bit <<= 1) {
+            const bool upper = lane & bit;  // the upper element of the pair takes (partner - own)
+#pragma unroll
+            for (int i = 0; i < NV; ++i) {
+                const float o = __shfl_xor_sync(0xffffffffu, r[i], bit);
+                r[i] = upper ? o - r[i] : r[i] + o;
+            }
+        }
+        if (hb >= 64) {
+#pragma unroll
+            for (int i = 0; i + 1 < NV; i += 2) {
+                const float a0 = r[i], a1 = r[i + 1];
+                r[i] = a0 + a1;
+                r[i + 1] = a0 - a1;
+            }
+        }
+        if (hb >= 128 && NV == 4) {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float a0 = r[i], a2 = r[i + 2];
+                r[i] = a0 + a2;
+                r[i + 2] = a0 - a2;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < NV; ++i) row[lane + 32 * i] = r[i] * nrm;
+    }
     __syncwarp();
 }
 
@@ -411,9 +437,14 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
         convert_k_scales<D>(krec, srK, rK, cK);
         __syncwarp();
 
-        // ---- q' B fragments (column part hl of head 4j + hq) and the group sums Q_g
+        // ---- q' B fragments (column part hl of head 4j + hq) and the group sums Q_g.
+        // Lanes g = 2hq and 2hq + 1 (lane ^ 4) need the same products, one the
+        // fp16 high part, the other the low part: each computes half the k-tiles
+        // (hl = 0 the first half) with both parts, keeps its own and passes its
+        // partner the other through one shuffle per register.
         uint32_t Bq[NTN][NKT][2];
         uint32_t BQ[NTN];
+        constexpr int HK = (NKT + 1) / 2;  // k-tiles per lane of the pair
 #pragma unroll
         for (int j = 0; j < NTN; ++j) {
             const int hh = 4 * j + hq;
@@ -422,23 +453,47 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
             float Qg[NG];
 #pragma unroll
             for (int g = 0; g < NG; ++g) Qg[g] = 0.f;
+            uint32_t own[HK][2], give[HK][2];
 #pragma unroll
-            for (int kt = 0; kt < NKT; ++kt) {
-                const int k = 16 * kt + 2 * tig;
+            for (int kk = 0; kk < HK; ++kk) {
+                const int kt = kk + (hl ? HK : 0);
+                const bool kv = kt < NKT;
+                const int k = 16 * (kv ? kt : 0) + 2 * tig;
                 const float2 q01 = *reinterpret_cast<const float2 *>(qh + k);
                 const float2 q89 = *reinterpret_cast<const float2 *>(qh + k + 8);
                 const float2 c01 = *reinterpret_cast<const float2 *>(cK + k);
                 const float2 c89 = *reinterpret_cast<const float2 *>(cK + k + 8);
-                const float2 v01 = __fmul2_rn(q01, c01), v89 = __fmul2_rn(q89, c89);
-                Qg[kt / 2] += (v01.x + v01.y) + (v89.x + v89.y);
+                const float2 v01 = __fmul2_rn(q01, c01);
                 // channels 8..15 of a k-tile sit at odd code positions (scale 2^-18): times 4
-                Bq[j][kt][0] = hv ? hilo_part(v01.x, v01.y, hl) : 0u;
-                Bq[j][kt][1] = hv ? hilo_part(v89.x * 4.f, v89.y * 4.f, hl) : 0u;
+                const float2 v89 = __fmul2_rn(__fmul2_rn(q89, c89), f2(4.f, 4.f));
+#pragma unroll
+                for (int g = 0; g < NG; ++g)
+                    if (kv && g == kt / 2) Qg[g] += (v01.x + v01.y) + 0.25f * (v89.x + v89.y);
+                uint32_t h0, l0, h1, l1;
+                split_hilo(v01.x, v01.y, h0, l0);
+                split_hilo(v89.x, v89.y, h1, l1);
+                own[kk][0] = hl ? l0 : h0;
+                own[kk][1] = hl ? l1 : h1;
+                give[kk][0] = hl ? h0 : l0;  // the partner's part of these products
+                give[kk][1] = hl ? h1 : l1;
+            }
+#pragma unroll
+            for (int kk = 0; kk < HK; ++kk) {
+                const uint32_t r0 = __shfl_xor_sync(0xffffffffu, give[kk][0], 4);
+                const uint32_t r1 = __shfl_xor_sync(0xffffffffu, give[kk][1], 4);
+                // k-tile kk is this lane's own when hl = 0, the partner's when hl = 1; k-tile HK + kk the reverse
+                Bq[j][kk][0] = hv ? (hl ? r0 : own[kk][0]) : 0u;
+                Bq[j][kk][1] = hv ? (hl ? r1 : own[kk][1]) : 0u;
+                if (HK + kk < NKT) {
+                    Bq[j][HK + kk][0] = hv ? (hl ? own[kk][0] : r0) : 0u;
+                    Bq[j][HK + kk][1] = hv ? (hl ? own[kk][1] : r1) : 0u;
+                }
             }
 #pragma unroll
             for (int g = 0; g < NG; ++g) {
                 Qg[g] += __shfl_xor_sync(0xffffffffu, Qg[g], 1);
                 Qg[g] += __shfl_xor_sync(0xffffffffu, Qg[g], 2);
+                Qg[g] += __shfl_xor_sync(0xffffffffu, Qg[g], 4);  // the pair's other half of the k-tiles
             }
             float q0 = 0.f, q1 = 0.f;
 #pragma unroll
@@ -599,8 +654,8 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
         __syncwarp();
         const float *rsV = scr, *rV = scr + NG * kBlockTokens, *cV = scr + (NG + 1) * kBlockTokens;
 
-        // ---- bias_{h,g} = sum_t p_t r_t m^V_{t,g} on the tensor cores
-        float accB[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---- bias_{h,g} = sum_t p_t r_t m^V_{t,g} on the tensor cores (two chains)
+        float accB[4] = {0.f, 0.f, 0.f, 0.f}, accB2[4] = {0.f, 0.f, 0.f, 0.f};
         {
             const __half *mh = reinterpret_cast<const __half *>(vrec + R::kMOff);
 #pragma unroll
@@ -618,9 +673,12 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
                     bb0 = *reinterpret_cast<uint32_t *>(&p0);
                     bb1 = *reinterpret_cast<uint32_t *>(&p1);
                 }
-                mma16816(accB, Ab, bb0, bb1);
+                if (ks & 1) mma16816(accB2, Ab, bb0, bb1);
+                else mma16816(accB, Ab, bb0, bb1);
             }
         }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) accB[i] += accB2[i];
         const float2 bpair = hilo_sum(accB);  // (h, groups 2tig, 2tig+1)
 
         // ---- P V, one group set at a time
@@ -652,43 +710,49 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
             const float bx = __shfl_sync(0xffffffffu, bpair.x, 4 * h + gsrc / 2);
             const float by = __shfl_sync(0xffffffffu, bpair.y, 4 * h + gsrc / 2);
             const float bias = ((gsrc & 1) ? by : bx) * kTwoM16;
-            // two 8-channel n-tiles at a time: independent MMA chains interleave
+            // two 8-channel n-tiles of every copy's group at a time: C x 2 independent
+            // MMA chains, interleaved token slice by token slice
 #pragma unroll
             for (int j4 = 0; j4 < kGroup / 8; j4 += 2) {
                 float mine[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                CodeWord vw[C][2][2];
+                float acc4[C][2][4];
 #pragma unroll
                 for (int cc = 0; cc < C; ++cc) {
                     const int gg = st * C + cc;
-                    if (gg >= NG) continue;
-                    const int nt0 = gg * (kGroup / 8) + j4;
-                    CodeWord vw[2][2];
-                    float acc4[2][4];
+                    const int nt0 = (gg < NG ? gg : 0) * (kGroup / 8) + j4;
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
                         const uint2 vw2 = reinterpret_cast<const uint2 *>(vrec)[(nt0 + jj) * 32 + lane];
-                        vw[jj][0] = CodeWord(vw2.x);
-                        vw[jj][1] = CodeWord(vw2.y);
-                        acc4[jj][0] = acc4[jj][1] = acc4[jj][2] = acc4[jj][3] = 0.f;
+                        vw[cc][jj][0] = CodeWord(vw2.x);
+                        vw[cc][jj][1] = CodeWord(vw2.y);
+                        acc4[cc][jj][0] = acc4[cc][jj][1] = acc4[cc][jj][2] = acc4[cc][jj][3] = 0.f;
                     }
+                }
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
+                for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+                    for (int cc = 0; cc < C; ++cc) {
+                        if (st * C + cc >= NG) continue;
 #pragma unroll
                         for (int jj = 0; jj < 2; ++jj) {
                             uint32_t bb[2];
 #pragma unroll
                             for (int cs = 0; cs < 2; ++cs) {
                                 const int m = 2 * ks + cs, am = m % 4;
-                                bb[cs] = code_pair(vw[jj][am / 2], 4 * (am % 2) + m / 4);
+                                bb[cs] = code_pair(vw[cc][jj][am / 2], 4 * (am % 2) + m / 4);
                             }
-                            mma16816(acc4[jj], Av[ks], bb[0], bb[1]);
+                            mma16816(acc4[cc][jj], Av[ks], bb[0], bb[1]);
                         }
                     }
-                    // the rows of this lane's copy carry the heads of group gg only when cc == copy
+                }
+                // the rows of this lane's copy carry the heads of group gg only when cc == copy
+#pragma unroll
+                for (int cc = 0; cc < C; ++cc)
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) mine[jj][i] = cc == copy ? acc4[jj][i] : mine[jj][i];
-                }
+                        for (int i = 0; i < 4; ++i) mine[jj][i] = cc == copy ? acc4[cc][jj][i] : mine[jj][i];
                 if (gv) {
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
@@ -897,8 +961,19 @@ __device__ void warp_merge(const DecodeArgs &a, int hb, DecWarpSmem<D, GRP> &sm,
 
 // Merge of one unit by all warps of the CTA (many partials).  Every thread
 // of the CTA calls it with the same arguments; the whole dynamic shared
-// memory is scratch.  A slot of a warp whose range is empty was never
-// written: it is neither read nor weighted.
+// memory is scratch.  The unit's block partials (slots wf + unit .. wl + unit,
+// contiguous) and its tail partial are copied into shared memory in one
+// round of asynchronous 16-byte copies; everything after that is shared-memory
+// arithmetic.  A slot of a warp whose range is empty was never written: it is
+// neither read nor weighted.
+template <int D, int GRP>
+struct CtaMergeLayout {
+    static constexpr int SR = slot_row<D>();
+    static constexpr int kSlot = GRP * SR;  // floats per partial
+    // parts [P][GRP][SR], tail [GRP][SR], then the small arrays
+    static __host__ __device__ constexpr size_t fixed_floats() { return kSlot + 4 * GRP + 2 * GRP * D; }
+};
+
 template <int D, int GRP, bool MQ>
 __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int unit, long long wf, long long wl,
                           long long total, long long nw)
@@ -906,113 +981,79 @@ __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int 
     constexpr int W = dec_warps<D, GRP>();
     constexpr int NT = W * 32;
     constexpr int SR = slot_row<D>();
-    constexpr int NQ = GRP * D / 4;  // float4 columns of a unit's output
-    constexpr int G = NT / NQ;       // partial groups summed in parallel
-    constexpr int UN = 8;            // partial loads in flight per thread
-    static_assert(G >= 1, "merge layout");
+    constexpr int SLOT = GRP * SR;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int P = (int)(wl - wf + 1);
-    const float *tl = a.tail_partials + (size_t)unit * GRP * SR;
-    const float *slots = a.partials + (size_t)(wf + unit) * GRP * SR;  // slot of warp wf + p at p * GRP * SR
+    float *parts = reinterpret_cast<float *>(smem);  // [P][GRP][SR]
+    float *tailp = parts + (size_t)P * SLOT;         // [GRP][SR]
+    float *Mh = tailp + SLOT;                        // [GRP]
+    float *Lh = Mh + GRP;                            // [GRP]
+    float *Wt = Lh + GRP;                            // [GRP] tail weight / L
+    float *Li = Wt + GRP;                            // [GRP] 1 / L
+    float *obuf = Li + GRP;                          // [GRP][D] block part (rotated, then un-rotated)
+    float *otl = obuf + GRP * D;                     // [GRP][D] tail part
+    float *wts = otl + GRP * D;                      // [P][GRP] weights exp2(m - M)
 
-    // scratch, every array starting on a 16-byte boundary
-    constexpr int SMALL = (W * GRP + 3 * GRP + 3) & ~3;      // red [W][GRP], Mh, Lh, Wt [GRP]
-    float4 *acc4 = reinterpret_cast<float4 *>(smem);         // [G][NQ]
-    float *obuf = reinterpret_cast<float *>(acc4 + G * NQ);  // [GRP][D]
-    float *otl = obuf + GRP * D;                             // [GRP][D]
-    float *red = otl + GRP * D;
-    float *Mh = red + W * GRP;
-    float *Lh = Mh + GRP;
-    float *Wt = Lh + GRP;
-    float2 *ml = reinterpret_cast<float2 *>(red + SMALL);    // [P][GRP] (m, l); m = -inf for an empty warp
-    float *wts = reinterpret_cast<float *>(ml + P * GRP);    // [P][GRP]
-
-    // (m, l) of every partial and head, and the maximum per head
-    const int hh = tid % GRP;  // NT is a multiple of 32, so every thread keeps one head
-    float mx = -INFINITY;
-    for (int idx = tid; idx < P * GRP; idx += NT) {
-        const long long w = wf + idx / GRP;
-        float2 v = f2(-INFINITY, 0.f);
-        if (part_begin(w, total, nw) < part_begin(w + 1, total, nw))
-            v = __ldcg(reinterpret_cast<const float2 *>(slots + (size_t)(idx / GRP) * GRP * SR + hh * SR));
-        ml[idx] = v;
-        mx = fmaxf(mx, v.x);
-    }
-    for (int o = GRP; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if (lane < GRP) red[warp * GRP + lane] = mx;
-    __syncthreads();
-    if (tid < GRP) {
-        float M = __ldcg(tl + tid * SR);
-        for (int w = 0; w < W; ++w) M = fmaxf(M, red[w * GRP + tid]);
-        Mh[tid] = M;
+    // ---- one round of copies: the P partials, then the tail partial
+    {
+        const float *src = a.partials + (size_t)(wf + unit) * SLOT;
+        const int n16 = P * SLOT / 4;  // SLOT is a multiple of 4 floats
+        for (int i = tid; i < n16 + SLOT / 4; i += NT) {
+            const float *g = i < n16 ? src + 4 * (size_t)i : a.tail_partials + (size_t)unit * SLOT + 4 * (i - n16);
+            const uint32_t d = smem_u32(parts + 4 * (size_t)i);  // tailp follows parts directly
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(g) : "memory");
+        }
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+        asm volatile("cp.async.wait_group 0;\n" ::: "memory");
     }
     __syncthreads();
-    // weights exp2(m - M) and the normaliser
-    const float M = Mh[hh];
-    float ls = 0.f;
-    for (int idx = tid; idx < P * GRP; idx += NT) {
-        const float2 v = ml[idx];
-        const float wgt = (M > -INFINITY && v.x > -INFINITY) ? exp2f(v.x - M) : 0.f;
-        wts[idx] = wgt;
-        ls = fmaf(v.y, wgt, ls);
-    }
-    for (int o = GRP; o < 32; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-    __syncthreads();  // every thread has read red and written wts
-    if (lane < GRP) red[warp * GRP + lane] = ls;
-    // the weighted sum of the o rows: threads over (group of partials, float4 column)
-    if (tid < G * NQ) {
-        const int q = tid % NQ, pg = tid / NQ;
-        const int h2 = q / (D / 4), d4 = q % (D / 4);
-        float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int p0 = pg; p0 < P; p0 += G * UN) {
-            float4 v[UN];
-            float wv[UN];
+    // ---- per head: the largest m, the weights and the normaliser (warp h for head h)
+    const bool all_valid = total >= nw;  // then every warp's range holds at least one item
+    for (int h = warp; h < GRP; h += W) {
+        float mx = -INFINITY;
+        for (int p = lane; p < P; p += 32) {
+            const long long w = wf + p;
+            if (all_valid || part_begin(w, total, nw) < part_begin(w + 1, total, nw))
+                mx = fmaxf(mx, parts[(size_t)p * SLOT + h * SR]);
+        }
 #pragma unroll
-            for (int u = 0; u < UN; ++u) {
-                const int p = p0 + u * G;
-                wv[u] = p < P ? wts[p * GRP + h2] : 0.f;
-                v[u] = wv[u] != 0.f ? __ldcg(reinterpret_cast<const float4 *>(slots + (size_t)p * GRP * SR + h2 * SR + 4) + d4)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float mt = tailp[h * SR];
+        const float M = fmaxf(mx, mt);
+        float ls = 0.f;
+        for (int p = lane; p < P; p += 32) {
+            const long long w = wf + p;
+            float wgt = 0.f;
+            if (M > -INFINITY && (all_valid || part_begin(w, total, nw) < part_begin(w + 1, total, nw))) {
+                const float m = parts[(size_t)p * SLOT + h * SR];
+                wgt = m > -INFINITY ? exp2f(m - M) : 0.f;
+                ls = fmaf(parts[(size_t)p * SLOT + h * SR + 1], wgt, ls);
             }
+            wts[p * GRP + h] = wgt;
+        }
 #pragma unroll
-            for (int u = 0; u < UN; ++u) {
-                s4.x = fmaf(v[u].x, wv[u], s4.x);
-                s4.y = fmaf(v[u].y, wv[u], s4.y);
-                s4.z = fmaf(v[u].z, wv[u], s4.z);
-                s4.w = fmaf(v[u].w, wv[u], s4.w);
-            }
+        for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+        if (lane == 0) {
+            const float wt = (M > -INFINITY && mt > -INFINITY) ? exp2f(mt - M) : 0.f;
+            const float L = fmaf(wt, tailp[h * SR + 1], ls);
+            const float li = L > 0.f ? 1.f / L : 0.f;
+            Mh[h] = M; Lh[h] = L; Li[h] = li; Wt[h] = wt * li;
         }
-        acc4[pg * NQ + q] = s4;
     }
     __syncthreads();
-    if (tid < GRP) {
-        const float Mt = Mh[tid];
-        const float wt = Mt > -INFINITY ? exp2f(__ldcg(tl + tid * SR) - Mt) : 0.f;
-        float L = wt * __ldcg(tl + tid * SR + 1);
-        for (int w = 0; w < W; ++w) L += red[w * GRP + tid];
-        Lh[tid] = L;
-        Wt[tid] = wt;
-    }
-    __syncthreads();
-    if (tid < NQ) {
-        const int h2 = tid / (D / 4), d4 = tid % (D / 4);
-        float4 s4 = acc4[tid];
-        for (int pg = 1; pg < G; ++pg) {
-            const float4 v = acc4[pg * NQ + tid];
-            s4.x += v.x; s4.y += v.y; s4.z += v.z; s4.w += v.w;
+    // ---- weighted sum of the block parts, and the scaled tail part
+    for (int i = tid; i < GRP * D; i += NT) {
+        const int h = i / D, c = i % D;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains
+        int p = 0;
+        for (; p + 3 < P; p += 4) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                acc[e] = fmaf(wts[(p + e) * GRP + h], parts[(size_t)(p + e) * SLOT + h * SR + 4 + c], acc[e]);
         }
-        const float L = Lh[h2];
-        const float linv = L > 0.f ? 1.f / L : 0.f;
-        *reinterpret_cast<float4 *>(obuf + h2 * D + 4 * d4) = make_float4(s4.x * linv, s4.y * linv, s4.z * linv,
-                                                                          s4.w * linv);
-        const float wt = Wt[h2];
-        float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (wt > 0.f) {
-            t4 = __ldcg(reinterpret_cast<const float4 *>(tl + h2 * SR + 4) + d4);
-            const float f = wt * linv;
-            t4.x *= f; t4.y *= f; t4.z *= f; t4.w *= f;
-        }
-        *reinterpret_cast<float4 *>(otl + h2 * D + 4 * d4) = t4;
+        for (; p < P; ++p) acc[0] = fmaf(wts[p * GRP + h], parts[(size_t)p * SLOT + h * SR + 4 + c], acc[0]);
+        obuf[i] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * Li[h];
+        otl[i] = Wt[h] != 0.f ? tailp[h * SR + 4 + c] * Wt[h] : 0.f;
     }
     __syncthreads();
     if (warp < GRP) warp_fwht<D>(obuf + warp * D, 1, hb);
@@ -1039,9 +1080,9 @@ template <int D, int GRP>
 __host__ __device__ constexpr int cta_merge_max()
 {
     constexpr int W = dec_warps<D, GRP>();
-    constexpr int NQ = GRP * D / 4, G = W * 32 / NQ;
-    constexpr int fixed = G * NQ * 16 + 2 * GRP * D * 4 + ((W * GRP + 3 * GRP + 3) & ~3) * 4;
-    return (int)((sizeof(DecWarpSmem<D, GRP>) * W - fixed) / (GRP * 12));
+    constexpr int SLOT = GRP * slot_row<D>();
+    constexpr size_t avail = sizeof(DecWarpSmem<D, GRP>) * W / sizeof(float);
+    return (int)((avail - CtaMergeLayout<D, GRP>::fixed_floats()) / (SLOT + GRP));
 }
 
 template <int D, int GRP, typename Tin, bool MQ>
@@ -1182,25 +1223,40 @@ decode_kernel(DecodeArgs a, int hb)
     // mark.  Only a unit covered by more than kWarpMergeMax warps (and at most
     // cta_merge_max) can carry one, and the CTA's contiguous range touches at most three of those (the
     // first, one covered whole by at least kWarpMergeMax + 1 of its W warps,
-    // the last), so thread 0 lists them and every thread walks the same list.
+    // the last), so four threads look them up and every thread walks the same list.
     __shared__ int merge_list[4];
     __shared__ int merge_count;
     __syncthreads();
     const long long c_begin = part_begin((long long)blockIdx.x * W, total, nw);
     const long long c_end = part_begin((long long)(blockIdx.x + 1) * W, total, nw);
-    if (threadIdx.x == 0) {
-        __threadfence();
-        int cnt = 0;
+    // Candidates: the units of the CTA's range that more than kWarpMergeMax warps
+    // covered; their tickets are read by one thread each, in parallel.
+    __shared__ int merge_flag[4];
+    if (threadIdx.x < 4) {
+        merge_flag[threadIdx.x] = -1;
         if (c_begin < c_end) {
             const long long u_first = c_begin / per_unit, u_last = (c_end - 1) / per_unit;
-            for (long long unit = u_first; unit <= u_last && cnt < 4; ++unit) {
-                const long long ibase = unit * per_unit;
+            long long unit = -1;
+            int k = 0;
+            for (long long u = u_first; u <= u_last; ++u) {  // the threadIdx.x-th candidate
+                const long long ibase = u * per_unit;
                 const long long span = part_owner(ibase + per_unit - 1, total, nw) - part_owner(ibase, total, nw) + 1;
-                if (span > kWarpMergeMax && span <= cta_merge_max<D, GRP>() &&
-                    __ldcg(a.tickets + unit) == (kMergeFlag | blockIdx.x))
-                    merge_list[cnt++] = (int)unit;
+                if (span > kWarpMergeMax && span <= cta_merge_max<D, GRP>()) {
+                    if (k == (int)threadIdx.x) { unit = u; break; }
+                    ++k;
+                }
+            }
+            if (unit >= 0) {
+                __threadfence();
+                if (__ldcg(a.tickets + unit) == (kMergeFlag | blockIdx.x)) merge_flag[threadIdx.x] = (int)unit;
             }
         }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int cnt = 0;
+        for (int k = 0; k < 4; ++k)
+            if (merge_flag[k] >= 0) merge_list[cnt++] = merge_flag[k];
         merge_count = cnt;
     }
     __syncthreads();
