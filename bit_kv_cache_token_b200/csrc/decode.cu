@@ -83,8 +83,14 @@ __host__ __device__ constexpr int dec_sets()
 template <int D, int GRP>
 __host__ __device__ constexpr int dec_warps()
 {
+    // Registers are reserved for warps in groups of four: 9 to 12 warps per
+    // SM all leave 168 registers a thread.  The 8-row instantiation needs
+    // more than that (it spills over 200 bytes at 168), so it runs 8 warps
+    // with up to 255 registers and no spills: 156 against 170 us for two
+    // query tokens at 32705 cached tokens (Qwen3-4B shapes, batch 8).
     constexpr int fit = (227 * 1024) / (int)sizeof(DecWarpSmem<D, GRP>);
-    return fit < 12 ? fit : 12;
+    constexpr int cap = GRP == 8 ? 8 : 12;
+    return fit < cap ? fit : cap;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
@@ -296,6 +302,24 @@ __device__ __forceinline__ long long part_owner(long long i, long long total, lo
 {
     return ((i + 1) * nw + total - 1) / total - 1;
 }
+
+// The block partials of one unit.  When every warp holds at least one item
+// (total >= nw) they are the slots of the contiguous warps wf .. wf + n - 1.
+// With fewer items than warps every warp holds at most one, so the unit's
+// per_unit items have per_unit distinct owners, spread over the grid; only
+// their slots were written, and only those are enumerated.
+struct UnitSlots {
+    long long ibase, wf, total, nw;
+    int n;  // partials
+    __device__ UnitSlots(long long unit, long long per_unit, long long total_, long long nw_)
+        : ibase(unit * per_unit), total(total_), nw(nw_)
+    {
+        wf = part_owner(ibase, total, nw);
+        n = total >= nw ? (int)(part_owner(ibase + per_unit - 1, total, nw) - wf + 1) : (int)per_unit;
+    }
+    // warp whose slot holds partial k
+    __device__ long long warp(int k) const { return total >= nw ? wf + k : part_owner(ibase + k, total, nw); }
+};
 
 // Element offset of row v (query v / heads_per_kv, head v % heads_per_kv) of
 // unit (sequence s, kv head hk) in q and out, laid out [S][num_queries][Hq][D].
@@ -895,27 +919,23 @@ __device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int u
     __syncwarp();
 }
 
-// Merge of one unit by a single warp (few partials): block partials from the
-// slots of warps [wf, wl] (empty ranges skipped), the tail partial, the
-// un-rotation, the output.  Uses the warp's record buffers as scratch.
+// Merge of one unit by a single warp (few partials): the unit's block
+// partials, the tail partial, the un-rotation, the output.  Uses the warp's
+// record buffers as scratch.
 template <int D, int GRP, bool MQ>
-__device__ void warp_merge(const DecodeArgs &a, int hb, DecWarpSmem<D, GRP> &sm, int unit, long long wf, long long wl,
-                           long long total, long long nw)
+__device__ void warp_merge(const DecodeArgs &a, int hb, DecWarpSmem<D, GRP> &sm, int unit, const UnitSlots &us)
 {
     constexpr int SR = slot_row<D>();
     const int lane = threadIdx.x & 31;
     const float *tl = a.tail_partials + (size_t)unit * GRP * SR;
     float *obuf = reinterpret_cast<float *>(sm.rec[0]);  // [GRP][D]
     float *otl = reinterpret_cast<float *>(sm.rec[1]);   // [GRP][D]
-    const int P = (int)(wl - wf + 1);
+    const int P = us.n;
     for (int hh = 0; hh < GRP; ++hh) {
         // lanes over partials: the maximum, then weights and the normaliser
         float M = -INFINITY;
-        for (int p = lane; p < P; p += 32) {
-            const long long w = wf + p;
-            if (part_begin(w, total, nw) < part_begin(w + 1, total, nw))
-                M = fmaxf(M, __ldcg(a.partials + (size_t)(w + unit) * GRP * SR + hh * SR));
-        }
+        for (int p = lane; p < P; p += 32)
+            M = fmaxf(M, __ldcg(a.partials + (size_t)(us.warp(p) + unit) * GRP * SR + hh * SR));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         const float mtl = __ldcg(tl + hh * SR);
@@ -925,9 +945,7 @@ __device__ void warp_merge(const DecodeArgs &a, int hb, DecWarpSmem<D, GRP> &sm,
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) acc[c] = 0.f;
         for (int p = 0; p < P; ++p) {
-            const long long w = wf + p;
-            if (!(part_begin(w, total, nw) < part_begin(w + 1, total, nw))) continue;
-            const float *row = a.partials + (size_t)(w + unit) * GRP * SR + hh * SR;
+            const float *row = a.partials + (size_t)(us.warp(p) + unit) * GRP * SR + hh * SR;
             const float m = __ldcg(row);
             const float wgt = M > -INFINITY ? exp2f(m - M) : 0.f;
             if (wgt == 0.f) continue;
@@ -975,15 +993,14 @@ struct CtaMergeLayout {
 };
 
 template <int D, int GRP, bool MQ>
-__device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int unit, long long wf, long long wl,
-                          long long total, long long nw)
+__device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int unit, const UnitSlots &us)
 {
     constexpr int W = dec_warps<D, GRP>();
     constexpr int NT = W * 32;
     constexpr int SR = slot_row<D>();
     constexpr int SLOT = GRP * SR;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int P = (int)(wl - wf + 1);
+    const int P = us.n;
     float *parts = reinterpret_cast<float *>(smem);  // [P][GRP][SR]
     float *tailp = parts + (size_t)P * SLOT;         // [GRP][SR]
     float *Mh = tailp + SLOT;                        // [GRP]
@@ -996,10 +1013,13 @@ __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int 
 
     // ---- one round of copies: the P partials, then the tail partial
     {
-        const float *src = a.partials + (size_t)(wf + unit) * SLOT;
         const int n16 = P * SLOT / 4;  // SLOT is a multiple of 4 floats
+        const bool contiguous = us.total >= us.nw;  // slots wf + unit .. wf + unit + P - 1
         for (int i = tid; i < n16 + SLOT / 4; i += NT) {
-            const float *g = i < n16 ? src + 4 * (size_t)i : a.tail_partials + (size_t)unit * SLOT + 4 * (i - n16);
+            const float *g;
+            if (i >= n16) g = a.tail_partials + (size_t)unit * SLOT + 4 * (i - n16);
+            else if (contiguous) g = a.partials + (size_t)(us.wf + unit) * SLOT + 4 * (size_t)i;
+            else g = a.partials + (size_t)(us.warp(i / (SLOT / 4)) + unit) * SLOT + 4 * (i % (SLOT / 4));
             const uint32_t d = smem_u32(parts + 4 * (size_t)i);  // tailp follows parts directly
             asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(g) : "memory");
         }
@@ -1008,23 +1028,17 @@ __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int 
     }
     __syncthreads();
     // ---- per head: the largest m, the weights and the normaliser (warp h for head h)
-    const bool all_valid = total >= nw;  // then every warp's range holds at least one item
     for (int h = warp; h < GRP; h += W) {
         float mx = -INFINITY;
-        for (int p = lane; p < P; p += 32) {
-            const long long w = wf + p;
-            if (all_valid || part_begin(w, total, nw) < part_begin(w + 1, total, nw))
-                mx = fmaxf(mx, parts[(size_t)p * SLOT + h * SR]);
-        }
+        for (int p = lane; p < P; p += 32) mx = fmaxf(mx, parts[(size_t)p * SLOT + h * SR]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         const float mt = tailp[h * SR];
         const float M = fmaxf(mx, mt);
         float ls = 0.f;
         for (int p = lane; p < P; p += 32) {
-            const long long w = wf + p;
             float wgt = 0.f;
-            if (M > -INFINITY && (all_valid || part_begin(w, total, nw) < part_begin(w + 1, total, nw))) {
+            if (M > -INFINITY) {
                 const float m = parts[(size_t)p * SLOT + h * SR];
                 wgt = m > -INFINITY ? exp2f(m - M) : 0.f;
                 ls = fmaf(parts[(size_t)p * SLOT + h * SR + 1], wgt, ls);
@@ -1207,10 +1221,9 @@ decode_kernel(DecodeArgs a, int hb)
         prev = __shfl_sync(0xffffffffu, prev, 0);
         if (prev + cnt == (uint32_t)per_unit) {
             __threadfence();
-            const long long wf = part_owner(ibase, total, nw), wl = part_owner(ibase + per_unit - 1, total, nw);
-            const long long span = wl - wf + 1;
-            if (span <= kWarpMergeMax || span > cta_merge_max<D, GRP>()) {
-                warp_merge<D, GRP, MQ>(a, hb, sm, unit, wf, wl, total, nw);
+            const UnitSlots us(unit, per_unit, total, nw);
+            if (us.n <= kWarpMergeMax || us.n > cta_merge_max<D, GRP>()) {
+                warp_merge<D, GRP, MQ>(a, hb, sm, unit, us);
                 if (lane == 0) a.tickets[unit] = 0u;
             } else if (lane == 0) {
                 atomicExch(a.tickets + unit, kMergeFlag | blockIdx.x);
@@ -1239,8 +1252,7 @@ decode_kernel(DecodeArgs a, int hb)
             long long unit = -1;
             int k = 0;
             for (long long u = u_first; u <= u_last; ++u) {  // the threadIdx.x-th candidate
-                const long long ibase = u * per_unit;
-                const long long span = part_owner(ibase + per_unit - 1, total, nw) - part_owner(ibase, total, nw) + 1;
+                const int span = UnitSlots(u, per_unit, total, nw).n;
                 if (span > kWarpMergeMax && span <= cta_merge_max<D, GRP>()) {
                     if (k == (int)threadIdx.x) { unit = u; break; }
                     ++k;
@@ -1263,9 +1275,7 @@ decode_kernel(DecodeArgs a, int hb)
     const int nmerge = merge_count;
     for (int j = 0; j < nmerge; ++j) {
         const int unit = merge_list[j];
-        const long long ibase = (long long)unit * per_unit;
-        const long long wf = part_owner(ibase, total, nw), wl = part_owner(ibase + per_unit - 1, total, nw);
-        cta_merge<D, GRP, MQ>(a, hb, smem_raw, unit, wf, wl, total, nw);
+        cta_merge<D, GRP, MQ>(a, hb, smem_raw, unit, UnitSlots(unit, per_unit, total, nw));
         if (threadIdx.x == 0) a.tickets[unit] = 0u;
     }
 }

@@ -52,6 +52,17 @@ def max_over_ranks(x: float, world: int, device: torch.device | str = "cpu") -> 
     return float(t.item())
 
 
+def gather_floats(x: float, world: int, device: torch.device | str = "cpu") -> list[float]:
+    """x of every rank, in rank order (every rank gets the list)."""
+    if world <= 1:
+        return [float(x)]
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    out = [torch.empty_like(t) for _ in range(world)]
+    dist.all_gather(out, t)
+    return [float(o.item()) for o in out]
+
+
 def rank_seed(base: int, rank: int) -> int:
     """Seed of a rank's synthetic batch: every rank draws a batch of its own."""
     return int(base) + 1000 * int(rank)
