@@ -237,9 +237,15 @@ __device__ __forceinline__ void stage_rows(const __nv_bfloat16 *rows, TcStage<D>
     asm volatile("cp.async.wait_group 0;\n" ::: "memory");
 }
 
-// Physical float4 slot of logical slot q in row `row` of a transpose buffer:
-// the eight lanes of one 16-byte read phase then hit distinct banks.
-__device__ __forceinline__ int xswz(int row, int q) { return q ^ ((((row >> 3) << 1) | (row & 1)) & 7); }
+// Physical float4 slot of logical slot q in row `row` (t = row >> 3, g =
+// row & 7) of a transpose buffer: q xor (t1 ^ g1, t0 ^ g0, g0).  A 16-byte
+// read phase (eight lanes: rows 8 t + g for t = 0..3 and two g differing in
+// bit 0) and an 8-byte write phase (sixteen lanes: rows 8 t + g for one t and
+// four g, two slots each) then both meet every bank once.
+__device__ __forceinline__ int xswz(int row, int q)
+{
+    return q ^ (((((row >> 4) ^ (row >> 1)) & 1) << 2) | ((((row >> 3) ^ row) & 1) << 1) | (row & 1));
+}
 
 // One warp's share of X H for a bf16 block: the 32 rotated channels of group j
 // (unnormalised: the stored r takes the 1/sqrt(HB)), all 128 tokens, into X
