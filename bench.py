@@ -49,7 +49,10 @@ QB_WORKLOAD = "Llama-3-8B-shaped bulk prefill quantise: 32 batch x 32 layers x 8
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one decode launch at context 32705 for this
 # batch, from one ncu capture of `bench.py --profile decode` with the current decode kernel; None whenever
 # the decode kernel has changed since the last capture.
-DECODE_TRAFFIC_BYTES = None
+DECODE_TRAFFIC_BYTES = 219994368 + 4283648
+# The same for one bulk-quantisation launch of `bench.py --profile quantize` (16 of the 1024 sequences); the
+# traffic grows with the sequences, so the full workload's is 64 times this.
+QUANT_TRAFFIC_BYTES_16SEQ = 537332992 + 97235968
 
 
 def _peaks():
@@ -927,7 +930,10 @@ def main():
         if q:
             line["quantize"] = {"workload": q["workload"], "gbs": q["gbs"], "ms": q["ms"], "frac": q["frac"],
                                 "algorithmic_bytes": q["bytes"], "peak": r["peak"], "status": q["status"],
-                                "roofline_alu": q["alu"]}
+                                "roofline_alu": q["alu"],
+                                "traffic": QUANT_TRAFFIC_BYTES_16SEQ * (QB_SEQS // 16) if not args.small else None,
+                                "traffic_source": "ncu capture of 16 sequences, scaled by 64 (traffic grows with the "
+                                                  "sequences)"}
         if r["ablation"]:
             line["ablation"] = r["ablation"]
         if r["multi"]:
