@@ -16,7 +16,7 @@
 //
 // B200 mapping.  The work of a launch is a list of items, unit by unit (a
 // unit is one (sequence, kv head)): the unit's max_tokens / 128 blocks, then
-// kTailSlots items for its residual tail.  Every warp of a persistent grid (one CTA
+// kTailSlots items for its residual tail, 32 tokens each.  Every warp of a persistent grid (one CTA
 // per SM) takes an equal contiguous range of that list, so the load is even
 // whatever the number of units and their lengths relative to the SM count.
 // Where a range crosses into a new unit the warp starts a new online softmax.
@@ -39,13 +39,14 @@
 // c * 2^-18.  The factor 4 between the two is folded into the other operand
 // (it depends only on the contracted index), the remaining 2^-16 into the
 // scales.  When the GQA group has fewer than 8 heads, the spare P V rows
-// carry copies of the heads working on other channel groups.  The tail item
-// is attended on CUDA cores with load-parallel loops.  Several query tokens
+// carry copies of the heads working on other channel groups.  A tail slot is
+// attended on CUDA cores and its output rotated, so that it merges like a
+// block partial.  Several query tokens
 // per sequence (MQ instantiations) are more rows on the same kv head, with a
 // causal limit applied in the last block and the tail.
 //
 // Merging.  Every (warp, unit) segment writes one partial (m, l, o_rot per
-// head); the tail item writes the unit's tail partial.  A per-unit ticket
+// head); every tail slot writes one more.  A per-unit ticket
 // counts the items whose partials are written; the warp that completes it
 // merges the unit itself when few warps covered it, and otherwise marks the
 // unit for its CTA, whose warps merge it together after they have all
@@ -337,14 +338,15 @@ __device__ __forceinline__ size_t qo_row(const DecodeArgs &a, int unit, int v)
 template <int D>
 __host__ __device__ constexpr int slot_row() { return D + 4; }
 
-// Partials are merged by the completing warp alone up to this many warps per unit.
-constexpr int kWarpMergeMax = 8;
-// Item slots of a unit's residual tail in the work list.  Attending up to 127
-// unrotated tokens on CUDA cores is a chain of dependent global loads, which
-// under the full streaming load costs about as much as three blocks; the
-// warp holding the first of these slots does it, the others have nothing to
-// do for them.
-constexpr int kTailSlots = 3;
+// Partials (block and tail) that the completing warp merges alone.
+constexpr int kWarpMergeMax = 12;
+// Item slots of a unit's residual tail in the work list: slot j stands for
+// tail tokens [32j, 32j + 32).  A warp attends the tokens of all the slots in
+// its range at once and writes their partial into the first (the others get
+// empty partials), so a long batch keeps one pass per tail while a short
+// one, whose items sit on separate warps, has the tail spread over up to four.
+constexpr int kTailSlots = kDecodeTailSlots;
+static_assert(kTailSlots * 32 >= kBlockTokens - 1, "the tail slots cover a tail of 127 tokens");
 // Marker of a unit whose merge the completing warp left to its CTA.
 constexpr uint32_t kMergeFlag = 0x80000000u;
 
@@ -798,73 +800,81 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
     return true;
 }
 
-// The residual tail of one unit: unrotated query, CUDA cores.  Writes the
-// tail partial (m, l, o per head, unrotated basis) to dst.  The tail is at
-// most 127 tokens and its cost is latency: every loop keeps a whole row (K)
-// or 16 rows (V) of loads in flight.
+// Tail tokens [t0, t1) of one unit (at most 127), attended by one warp with
+// the unrotated query on CUDA cores: lanes over tokens for the scores (a
+// whole row's loads issued together), over channel quads for P V (VB rows'
+// loads in flight).  The output is rotated before it is stored, so that the
+// partial (m, l, o per head) is in the basis of the block partials and
+// merges with them alike.  Runs after the segment's blocks: the record
+// buffers and the query buffer are scratch.
 template <int D, int GRP, typename Tin, bool MQ>
-__device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int unit, int ntail, int tlim0, float *dst)
+__device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int unit, int t0, int t1, int tlim0,
+                             int hb, float *dst)
 {
     constexpr int SR = slot_row<D>();
     constexpr int VB = 16;  // V rows per batch of loads
     const int lane = threadIdx.x & 31;
-    float *ps = reinterpret_cast<float *>(sm.rec[0]);  // [128][GRP] scores, then weights
-    float *qt = ps + kBlockTokens * GRP;               // [GRP][D] query, scaled (uniform reads: broadcasts)
-    static_assert(sizeof(float) * (kBlockTokens * GRP + GRP * D) <= sizeof(sm.rec), "tail scratch");
-    if constexpr (MQ) {
+    float *ps = reinterpret_cast<float *>(sm.rec[0]);  // [128][GRP] scores, then weights (index t - t0), both buffers
+    float *qt = &sm.qbuf[0][0];                        // [GRP][D] query, scaled (uniform reads: broadcasts)
+    float *ob = qt;                                    // [GRP][D] output, rotated in place (once the scores are done)
+    static_assert(sizeof(float) * kBlockTokens * GRP <= sizeof(sm.rec), "tail scratch");
+    const int nt = t1 - t0;
+    if (nt > 0) {
+        if constexpr (MQ) {
 #pragma unroll
-        for (int v = 0; v < GRP; ++v) {
-            const Tin *qv = static_cast<const Tin *>(a.q) + qo_row<D, GRP, MQ>(a, unit, v);
-            for (int d = lane; d < D; d += 32) qt[v * D + d] = In<Tin>::load1(qv + d) * a.scale_log2;
-        }
-    } else {
-        const Tin *qg = static_cast<const Tin *>(a.q) + (size_t)unit * GRP * D;
-        for (int i = lane; i < GRP * D; i += 32) qt[i] = In<Tin>::load1(qg + i) * a.scale_log2;
-    }
-    __syncwarp();
-    // scores: lanes over tokens, a row's loads issued together
-    const Tin *kt = static_cast<const Tin *>(a.k_tail) + (size_t)unit * kBlockTokens * D;
-    for (int t0 = 0; t0 < ntail; t0 += 32) {
-        const int t = t0 + lane;
-        if (t < ntail) {
-            float acc[GRP];
-#pragma unroll
-            for (int hh = 0; hh < GRP; ++hh) acc[hh] = 0.f;
-            float kv[D];
-#pragma unroll
-            for (int c8 = 0; c8 < D; c8 += 8) {
-                float k8[8];
-                In<Tin>::load8(kt + (size_t)t * D + c8, k8);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) kv[c8 + e] = k8[e];
+            for (int v = 0; v < GRP; ++v) {
+                const Tin *qv = static_cast<const Tin *>(a.q) + qo_row<D, GRP, MQ>(a, unit, v);
+                for (int d = lane; d < D; d += 32) qt[v * D + d] = In<Tin>::load1(qv + d) * a.scale_log2;
             }
+        } else {
+            const Tin *qg = static_cast<const Tin *>(a.q) + (size_t)unit * GRP * D;
+            for (int i = lane; i < GRP * D; i += 32) qt[i] = In<Tin>::load1(qg + i) * a.scale_log2;
+        }
+        __syncwarp();
+        // scores: lanes over tokens, a row's loads issued together
+        const Tin *kt = static_cast<const Tin *>(a.k_tail) + (size_t)unit * kBlockTokens * D;
+        for (int u0 = 0; u0 < nt; u0 += 32) {
+            const int u = u0 + lane, t = t0 + u;
+            if (u < nt) {
+                float acc[GRP];
 #pragma unroll
-            for (int c4 = 0; c4 < D; c4 += 4) {
+                for (int hh = 0; hh < GRP; ++hh) acc[hh] = 0.f;
+                float kv[D];
 #pragma unroll
-                for (int hh = 0; hh < GRP; ++hh) {
-                    const float4 qv = *reinterpret_cast<const float4 *>(qt + hh * D + c4);
-                    acc[hh] = fmaf(qv.x, kv[c4], acc[hh]);
-                    acc[hh] = fmaf(qv.y, kv[c4 + 1], acc[hh]);
-                    acc[hh] = fmaf(qv.z, kv[c4 + 2], acc[hh]);
-                    acc[hh] = fmaf(qv.w, kv[c4 + 3], acc[hh]);
+                for (int c8 = 0; c8 < D; c8 += 8) {
+                    float k8[8];
+                    In<Tin>::load8(kt + (size_t)t * D + c8, k8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) kv[c8 + e] = k8[e];
                 }
-            }
-            // several queries: row hh sees tail tokens t <= tlim0 + hh / heads_per_kv
 #pragma unroll
-            for (int hh = 0; hh < GRP; ++hh)
-                ps[t * GRP + hh] = (!MQ || t <= tlim0 + hh / a.heads_per_kv) ? acc[hh] : -INFINITY;
+                for (int c4 = 0; c4 < D; c4 += 4) {
+#pragma unroll
+                    for (int hh = 0; hh < GRP; ++hh) {
+                        const float4 qv = *reinterpret_cast<const float4 *>(qt + hh * D + c4);
+                        acc[hh] = fmaf(qv.x, kv[c4], acc[hh]);
+                        acc[hh] = fmaf(qv.y, kv[c4 + 1], acc[hh]);
+                        acc[hh] = fmaf(qv.z, kv[c4 + 2], acc[hh]);
+                        acc[hh] = fmaf(qv.w, kv[c4 + 3], acc[hh]);
+                    }
+                }
+                // several queries: row hh sees tail tokens t <= tlim0 + hh / heads_per_kv
+#pragma unroll
+                for (int hh = 0; hh < GRP; ++hh)
+                    ps[u * GRP + hh] = (!MQ || t <= tlim0 + hh / a.heads_per_kv) ? acc[hh] : -INFINITY;
+            }
         }
+        __syncwarp();
     }
-    __syncwarp();
-    // softmax over the tail tokens, lanes over tokens
+    // softmax over the range, lanes over tokens
     float mt[GRP], lt[GRP];
 #pragma unroll
     for (int hh = 0; hh < GRP; ++hh) {
         float sv[4], mx = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int t = lane + 32 * j;
-            sv[j] = t < ntail ? ps[t * GRP + hh] : -INFINITY;
+            const int u = lane + 32 * j;
+            sv[j] = u < nt ? ps[u * GRP + hh] : -INFINITY;
             mx = fmaxf(mx, sv[j]);
         }
 #pragma unroll
@@ -872,14 +882,14 @@ __device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int u
         float sum = 0.f;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int t = lane + 32 * j;
-            const float p = (t < ntail && (!MQ || sv[j] > -INFINITY)) ? exp2f(sv[j] - mx) : 0.f;
-            if (t < ntail) ps[t * GRP + hh] = p;
+            const int u = lane + 32 * j;
+            const float p = sv[j] > -INFINITY ? exp2f(sv[j] - mx) : 0.f;
+            if (u < nt) ps[u * GRP + hh] = p;
             sum += p;
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        mt[hh] = ntail > 0 ? mx : -INFINITY;
+        mt[hh] = mx;
         lt[hh] = sum;
     }
     __syncwarp();
@@ -890,18 +900,18 @@ __device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int u
     float4 o[GRP];
 #pragma unroll
     for (int hh = 0; hh < GRP; ++hh) o[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int t0 = 0; t0 < ntail; t0 += VB) {
+    for (int u0 = 0; u0 < nt; u0 += VB) {
         typename In<Tin>::Raw4 vr[VB];
 #pragma unroll
         for (int u = 0; u < VB; ++u)
-            vr[u] = In<Tin>::load4_raw(vt + (size_t)min(t0 + u, ntail - 1) * D + (act ? c0 : 0));
+            vr[u] = In<Tin>::load4_raw(vt + (size_t)(t0 + min(u0 + u, nt - 1)) * D + (act ? c0 : 0));
 #pragma unroll
         for (int u = 0; u < VB; ++u) {
-            if (act && t0 + u < ntail) {
+            if (act && u0 + u < nt) {
                 const float4 vv = In<Tin>::widen4(vr[u]);
 #pragma unroll
                 for (int hh = 0; hh < GRP; ++hh) {
-                    const float p = ps[(t0 + u) * GRP + hh];
+                    const float p = ps[(u0 + u) * GRP + hh];
                     o[hh].x = fmaf(p, vv.x, o[hh].x);
                     o[hh].y = fmaf(p, vv.y, o[hh].y);
                     o[hh].z = fmaf(p, vv.z, o[hh].z);
@@ -910,57 +920,73 @@ __device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int u
             }
         }
     }
+    // into the rotated basis of the block partials
+#pragma unroll
+    for (int hh = 0; hh < GRP; ++hh)
+        if (act) *reinterpret_cast<float4 *>(ob + hh * D + c0) = o[hh];
+    __syncwarp();
+    warp_fwht<D>(ob, GRP, hb);
 #pragma unroll
     for (int hh = 0; hh < GRP; ++hh) {
         float *row = dst + hh * SR;
         if (lane == 0) { row[0] = mt[hh]; row[1] = lt[hh]; }
-        if (act) *reinterpret_cast<float4 *>(row + 4 + c0) = o[hh];
+        if (act) *reinterpret_cast<float4 *>(row + 4 + c0) = *reinterpret_cast<const float4 *>(ob + hh * D + c0);
     }
     __syncwarp();
 }
 
-// Merge of one unit by a single warp (few partials): the unit's block
-// partials, the tail partial, the un-rotation, the output.  Uses the warp's
-// record buffers as scratch.
+// An empty partial (m = -inf, l = 0, o = 0) for GRP heads.
+template <int D, int GRP>
+__device__ __forceinline__ void empty_partial(float *dst)
+{
+    constexpr int SR = slot_row<D>();
+    const int lane = threadIdx.x & 31;
+    for (int i = lane; i < GRP * SR; i += 32) dst[i] = (i % SR == 0) ? -INFINITY : 0.f;
+}
+
+// Partial p of a unit: its block partials (p < us.n, in the slots of the
+// warps that hold its items), then its kTailSlots tail partials.  All are in
+// the rotated basis, and all were written (an empty one has m = -inf, l = 0).
+template <int D, int GRP>
+__device__ __forceinline__ const float *unit_partial(const DecodeArgs &a, int unit, const UnitSlots &us, int p)
+{
+    constexpr int SLOT = GRP * slot_row<D>();
+    return p < us.n ? a.partials + (size_t)(us.warp(p) + unit) * SLOT
+                    : a.tail_partials + ((size_t)unit * kTailSlots + (p - us.n)) * SLOT;
+}
+
+// Merge of one unit by a single warp (few partials): the log-sum-exp merge of
+// its partials, the un-rotation, the output.  Uses the warp's record buffers
+// as scratch.
 template <int D, int GRP, bool MQ>
 __device__ void warp_merge(const DecodeArgs &a, int hb, DecWarpSmem<D, GRP> &sm, int unit, const UnitSlots &us)
 {
     constexpr int SR = slot_row<D>();
     const int lane = threadIdx.x & 31;
-    const float *tl = a.tail_partials + (size_t)unit * GRP * SR;
     float *obuf = reinterpret_cast<float *>(sm.rec[0]);  // [GRP][D]
-    float *otl = reinterpret_cast<float *>(sm.rec[1]);   // [GRP][D]
-    const int P = us.n;
+    const int P = us.n + kTailSlots;
     for (int hh = 0; hh < GRP; ++hh) {
         // lanes over partials: the maximum, then weights and the normaliser
         float M = -INFINITY;
-        for (int p = lane; p < P; p += 32)
-            M = fmaxf(M, __ldcg(a.partials + (size_t)(us.warp(p) + unit) * GRP * SR + hh * SR));
+        for (int p = lane; p < P; p += 32) M = fmaxf(M, __ldcg(unit_partial<D, GRP>(a, unit, us, p) + hh * SR));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        const float mtl = __ldcg(tl + hh * SR);
-        M = fmaxf(M, mtl);
         float L = 0.f;
         float acc[D / 32];
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) acc[c] = 0.f;
         for (int p = 0; p < P; ++p) {
-            const float *row = a.partials + (size_t)(us.warp(p) + unit) * GRP * SR + hh * SR;
+            const float *row = unit_partial<D, GRP>(a, unit, us, p) + hh * SR;
             const float m = __ldcg(row);
-            const float wgt = M > -INFINITY ? exp2f(m - M) : 0.f;
+            const float wgt = (M > -INFINITY && m > -INFINITY) ? exp2f(m - M) : 0.f;
             if (wgt == 0.f) continue;
             L = fmaf(__ldcg(row + 1), wgt, L);
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) acc[c] = fmaf(__ldcg(row + 4 + 32 * c + lane), wgt, acc[c]);
         }
-        const float wt = M > -INFINITY ? exp2f(mtl - M) : 0.f;
-        L = fmaf(__ldcg(tl + hh * SR + 1), wt, L);
         const float linv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-            obuf[hh * D + 32 * c + lane] = acc[c] * linv;
-            otl[hh * D + 32 * c + lane] = wt > 0.f ? __ldcg(tl + hh * SR + 4 + 32 * c + lane) * wt * linv : 0.f;
-        }
+        for (int c = 0; c < D / 32; ++c) obuf[hh * D + 32 * c + lane] = acc[c] * linv;
     }
     __syncwarp();
     warp_fwht<D>(obuf, GRP, hb);
@@ -968,28 +994,26 @@ __device__ void warp_merge(const DecodeArgs &a, int hb, DecWarpSmem<D, GRP> &sm,
 #pragma unroll
         for (int v = 0; v < GRP; ++v) {
             float *ov = a.out + qo_row<D, GRP, MQ>(a, unit, v);
-            for (int d = lane; d < D; d += 32) ov[d] = obuf[v * D + d] + otl[v * D + d];
+            for (int d = lane; d < D; d += 32) ov[d] = obuf[v * D + d];
         }
     } else {
         float *out = a.out + (size_t)unit * GRP * D;
-        for (int i = lane; i < GRP * D; i += 32) out[i] = obuf[i] + otl[i];
+        for (int i = lane; i < GRP * D; i += 32) out[i] = obuf[i];
     }
     __syncwarp();
 }
 
 // Merge of one unit by all warps of the CTA (many partials).  Every thread
 // of the CTA calls it with the same arguments; the whole dynamic shared
-// memory is scratch.  The unit's block partials (slots wf + unit .. wl + unit,
-// contiguous) and its tail partial are copied into shared memory in one
-// round of asynchronous 16-byte copies; everything after that is shared-memory
-// arithmetic.  A slot of a warp whose range is empty was never written: it is
-// neither read nor weighted.
+// memory is scratch.  The unit's partials (block partials, then tail
+// partials) are copied into shared memory in one round of asynchronous
+// 16-byte copies; everything after that is shared-memory arithmetic.
 template <int D, int GRP>
 struct CtaMergeLayout {
     static constexpr int SR = slot_row<D>();
     static constexpr int kSlot = GRP * SR;  // floats per partial
-    // parts [P][GRP][SR], tail [GRP][SR], then the small arrays
-    static __host__ __device__ constexpr size_t fixed_floats() { return kSlot + 4 * GRP + 2 * GRP * D; }
+    // parts [P][GRP][SR], obuf [GRP][D], then 1/L and M per head (padded), then the weights [P][GRP]
+    static __host__ __device__ constexpr size_t fixed_floats() { return GRP * D + 2 * ((GRP + 3) / 4 * 4); }
 };
 
 template <int D, int GRP, bool MQ>
@@ -999,28 +1023,25 @@ __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int 
     constexpr int NT = W * 32;
     constexpr int SR = slot_row<D>();
     constexpr int SLOT = GRP * SR;
+    constexpr int GP = (GRP + 3) / 4 * 4;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int P = us.n;
+    const int P = us.n + kTailSlots;
     float *parts = reinterpret_cast<float *>(smem);  // [P][GRP][SR]
-    float *tailp = parts + (size_t)P * SLOT;         // [GRP][SR]
-    float *Mh = tailp + SLOT;                        // [GRP]
-    float *Lh = Mh + GRP;                            // [GRP]
-    float *Wt = Lh + GRP;                            // [GRP] tail weight / L
-    float *Li = Wt + GRP;                            // [GRP] 1 / L
-    float *obuf = Li + GRP;                          // [GRP][D] block part (rotated, then un-rotated)
-    float *otl = obuf + GRP * D;                     // [GRP][D] tail part
-    float *wts = otl + GRP * D;                      // [P][GRP] weights exp2(m - M)
+    float *obuf = parts + (size_t)P * SLOT;          // [GRP][D] block part (rotated, then un-rotated)
+    float *Li = obuf + GRP * D;                      // [GRP] 1 / L
+    float *Mh = Li + GP;                             // [GRP]
+    float *wts = Mh + GP;                            // [P][GRP] weights exp2(m - M)
 
-    // ---- one round of copies: the P partials, then the tail partial
+    // ---- one round of copies: the block partials, then the tail partials
     {
-        const int n16 = P * SLOT / 4;  // SLOT is a multiple of 4 floats
-        const bool contiguous = us.total >= us.nw;  // slots wf + unit .. wf + unit + P - 1
-        for (int i = tid; i < n16 + SLOT / 4; i += NT) {
+        const int nb16 = us.n * SLOT / 4, n16 = P * SLOT / 4;  // SLOT is a multiple of 4 floats
+        const bool contiguous = us.total >= us.nw;  // block partials in slots wf + unit .. wf + unit + n - 1
+        for (int i = tid; i < n16; i += NT) {
             const float *g;
-            if (i >= n16) g = a.tail_partials + (size_t)unit * SLOT + 4 * (i - n16);
+            if (i >= nb16) g = a.tail_partials + (size_t)unit * kTailSlots * SLOT + 4 * (size_t)(i - nb16);
             else if (contiguous) g = a.partials + (size_t)(us.wf + unit) * SLOT + 4 * (size_t)i;
             else g = a.partials + (size_t)(us.warp(i / (SLOT / 4)) + unit) * SLOT + 4 * (i % (SLOT / 4));
-            const uint32_t d = smem_u32(parts + 4 * (size_t)i);  // tailp follows parts directly
+            const uint32_t d = smem_u32(parts + 4 * (size_t)i);
             asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(g) : "memory");
         }
         asm volatile("cp.async.commit_group;\n" ::: "memory");
@@ -1033,29 +1054,23 @@ __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int 
         for (int p = lane; p < P; p += 32) mx = fmaxf(mx, parts[(size_t)p * SLOT + h * SR]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const float mt = tailp[h * SR];
-        const float M = fmaxf(mx, mt);
+        const float M = mx;
         float ls = 0.f;
         for (int p = lane; p < P; p += 32) {
-            float wgt = 0.f;
-            if (M > -INFINITY) {
-                const float m = parts[(size_t)p * SLOT + h * SR];
-                wgt = m > -INFINITY ? exp2f(m - M) : 0.f;
-                ls = fmaf(parts[(size_t)p * SLOT + h * SR + 1], wgt, ls);
-            }
+            const float m = parts[(size_t)p * SLOT + h * SR];
+            const float wgt = (M > -INFINITY && m > -INFINITY) ? exp2f(m - M) : 0.f;
+            ls = fmaf(parts[(size_t)p * SLOT + h * SR + 1], wgt, ls);
             wts[p * GRP + h] = wgt;
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
         if (lane == 0) {
-            const float wt = (M > -INFINITY && mt > -INFINITY) ? exp2f(mt - M) : 0.f;
-            const float L = fmaf(wt, tailp[h * SR + 1], ls);
-            const float li = L > 0.f ? 1.f / L : 0.f;
-            Mh[h] = M; Lh[h] = L; Li[h] = li; Wt[h] = wt * li;
+            Mh[h] = M;
+            Li[h] = ls > 0.f ? 1.f / ls : 0.f;
         }
     }
     __syncthreads();
-    // ---- weighted sum of the block parts, and the scaled tail part
+    // ---- weighted sum of the partials (an empty partial has weight 0 and zero rows)
     for (int i = tid; i < GRP * D; i += NT) {
         const int h = i / D, c = i % D;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains
@@ -1067,7 +1082,6 @@ __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int 
         }
         for (; p < P; ++p) acc[0] = fmaf(wts[p * GRP + h], parts[(size_t)p * SLOT + h * SR + 4 + c], acc[0]);
         obuf[i] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * Li[h];
-        otl[i] = Wt[h] != 0.f ? tailp[h * SR + 4 + c] * Wt[h] : 0.f;
     }
     __syncthreads();
     if (warp < GRP) warp_fwht<D>(obuf + warp * D, 1, hb);
@@ -1075,14 +1089,12 @@ __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int 
     if constexpr (MQ) {
         if (tid < GRP * (D / 4)) {  // a float4 of one row per thread
             const int v = tid / (D / 4), d4 = tid % (D / 4);
-            const float4 x = *reinterpret_cast<const float4 *>(obuf + v * D + 4 * d4);
-            const float4 y = *reinterpret_cast<const float4 *>(otl + v * D + 4 * d4);
             *reinterpret_cast<float4 *>(a.out + qo_row<D, GRP, MQ>(a, unit, v) + 4 * d4) =
-                make_float4(x.x + y.x, x.y + y.y, x.z + y.z, x.w + y.w);
+                *reinterpret_cast<const float4 *>(obuf + v * D + 4 * d4);
         }
     } else {
         float *out = a.out + (size_t)unit * GRP * D;
-        for (int i = tid; i < GRP * D; i += NT) out[i] = obuf[i] + otl[i];
+        for (int i = tid; i < GRP * D; i += NT) out[i] = obuf[i];
     }
     __syncthreads();  // the scratch is free again
 }
@@ -1147,7 +1159,6 @@ decode_kernel(DecodeArgs a, int hb)
         const int b0 = (int)(i - ibase);
         const int b1 = (int)min(seg_end - ibase, (long long)nb_max);
         const int b1r = min(b1, nblk);  // blocks beyond the sequence's length are skipped
-        const bool has_tail = i - ibase <= nb_max && seg_end - ibase > nb_max;
 
         float m_run[NTN], l_run[NTN];
 #pragma unroll
@@ -1208,9 +1219,15 @@ decode_kernel(DecodeArgs a, int hb)
                         *reinterpret_cast<float2 *>(pp + 4 + 8 * (g * (kGroup / 8) + jn) + 2 * tig) = orun[st][jn];
             }
         }
-        if (has_tail)
-            tail_partial<D, GRP, Tin, MQ>(a, sm, unit, ntail, n - a.num_queries - nblk * kBlockTokens,
-                                      a.tail_partials + (size_t)unit * GRP * SR);
+        // its tail slots [j0, j1): one pass over their tokens into slot j0's partial, the others empty
+        // (a warp with several slots attends their tokens at once; single slots spread a short batch's tail)
+        const long long j0 = max(i - ibase - nb_max, 0ll), j1 = seg_end - ibase - nb_max;
+        if (j0 < j1) {
+            float *tp = a.tail_partials + (size_t)unit * kTailSlots * GRP * SR;
+            tail_partial<D, GRP, Tin, MQ>(a, sm, unit, min(32 * (int)j0, ntail), min(32 * (int)j1, ntail),
+                                          n - a.num_queries - nblk * kBlockTokens, hb, tp + j0 * GRP * SR);
+            for (long long j = j0 + 1; j < j1; ++j) empty_partial<D, GRP>(tp + j * GRP * SR);
+        }
 
         // ---- arrival: this segment's items are done
         __syncwarp();
@@ -1222,7 +1239,8 @@ decode_kernel(DecodeArgs a, int hb)
         if (prev + cnt == (uint32_t)per_unit) {
             __threadfence();
             const UnitSlots us(unit, per_unit, total, nw);
-            if (us.n <= kWarpMergeMax || us.n > cta_merge_max<D, GRP>()) {
+            const int np = us.n + kTailSlots;  // partials to merge
+            if (np <= kWarpMergeMax || np > cta_merge_max<D, GRP>()) {
                 warp_merge<D, GRP, MQ>(a, hb, sm, unit, us);
                 if (lane == 0) a.tickets[unit] = 0u;
             } else if (lane == 0) {
@@ -1252,8 +1270,8 @@ decode_kernel(DecodeArgs a, int hb)
             long long unit = -1;
             int k = 0;
             for (long long u = u_first; u <= u_last; ++u) {  // the threadIdx.x-th candidate
-                const int span = UnitSlots(u, per_unit, total, nw).n;
-                if (span > kWarpMergeMax && span <= cta_merge_max<D, GRP>()) {
+                const int np = UnitSlots(u, per_unit, total, nw).n + kTailSlots;
+                if (np > kWarpMergeMax && np <= cta_merge_max<D, GRP>()) {
                     if (k == (int)threadIdx.x) { unit = u; break; }
                     ++k;
                 }

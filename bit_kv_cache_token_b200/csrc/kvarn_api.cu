@@ -106,8 +106,8 @@ size_t kvarn_decode_workspace_bytes(const kvarn_config *cfg, int num_q_heads)
     const int grp = num_q_heads / cfg->num_kv_heads;
     const size_t sh = (size_t)cfg->num_seqs * cfg->num_kv_heads;
     const size_t warps = (size_t)num_sms() * decode_warps_per_cta(cfg->head_dim, grp);
-    // tickets, one block partial per (warp, unit) segment (at most warps + units), one tail partial per unit
-    return ticket_bytes(cfg) + (warps + 2 * sh) * decode_slot_bytes(cfg->head_dim, grp);
+    // tickets, one block partial per (warp, unit) segment (at most warps + units), the tail slots' partials
+    return ticket_bytes(cfg) + (warps + sh * (1 + kDecodeTailSlots)) * decode_slot_bytes(cfg->head_dim, grp);
 }
 
 int kvarn_quantize_blocks(const kvarn_config *cfg, const void *k, const void *v, int num_tokens,

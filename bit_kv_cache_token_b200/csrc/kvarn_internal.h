@@ -43,7 +43,7 @@ struct DecodeArgs {
     int32_t *status;
     float *out;                 // [S][Hq][D]
     float *partials;            // [warps + units][grp][D+4]: one per (warp, unit) segment, at warp + unit
-    float *tail_partials;       // [units][grp][D+4]
+    float *tail_partials;       // [units][kDecodeTailSlots][grp][D+4]
     uint32_t *tickets;          // [units], zero between calls
     float scale_log2;           // softmax scale * log2(e)
     int num_kv_heads, grp, max_blocks, max_tokens;
@@ -72,6 +72,9 @@ cudaError_t run_append(const kvarn_config &c, const AppendArgs &a, cudaStream_t 
 cudaError_t run_dequantize(const kvarn_config &c, const DequantArgs &a, cudaStream_t st);
 cudaError_t run_decode(const kvarn_config &c, const DecodeArgs &a, int ctas, cudaStream_t st);
 cudaError_t run_set_length(int32_t *n_tokens, int num_seqs, int value, cudaStream_t st);
+
+// Item slots of a unit's residual tail in the decode work list, 32 tokens each.
+constexpr int kDecodeTailSlots = 4;
 
 // Warps per decode CTA (one CTA per SM by shared memory).
 int decode_warps_per_cta(int head_dim, int grp);

@@ -42,9 +42,9 @@ def test_workspace_bytes():
     cfg = kvarn.Config(8, 8, 128, 256)
     ws = kvarn.decode_workspace_bytes(cfg, 32)
     # tickets (64 units, padded to 256 B) + one partial per (warp, unit) segment, at most 148 SMs x 12 warps
-    # + 64, + one tail partial per unit; a partial is 4 heads x (m, l, pad, pad, o[128]) fp32.  Without a GPU
-    # the library assumes 148 SMs.
-    assert ws == 256 + (148 * 12 + 2 * 64) * 4 * 132 * 4
+    # + 64, + four tail-slot partials per unit; a partial is 4 heads x (m, l, pad, pad, o[128]) fp32.  Without a
+    # GPU the library assumes 148 SMs.
+    assert ws == 256 + (148 * 12 + 64 + 4 * 64) * 4 * 132 * 4
     assert kvarn.decode_workspace_bytes(cfg, 12) == 0  # not a multiple of the kv heads
 
 
