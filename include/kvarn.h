@@ -145,7 +145,8 @@ KVARN_API size_t kvarn_cache_bytes(const kvarn_config *cfg, int part);
  * on the current device: merge tickets (one uint32 per (sequence, kv head),
  * padded to 256 bytes), then partial results -- one per (warp, sequence x kv
  * head) segment of the persistent grid (at most SMs x warps per CTA + units)
- * and one per unit for its residual tail, each grp x (D + 4) fp32.  The size
+ * and four per unit for the slots of its residual tail, each grp x (D + 4)
+ * fp32.  The size
  * depends on the device's SM count: query it on the device that runs the
  * decode.  Zero the workspace once (e.g. cudaMemsetAsync) before its first
  * use; every decode call leaves the tickets zero again, so one workspace
