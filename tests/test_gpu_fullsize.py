@@ -113,3 +113,18 @@ def test_qwen_decode_at_checkpoint_contexts(total, layer):
 def test_phi_mha_decode_layer_16k_sampled():
     print("max abs err", _decode_layer(16, 32, 32, 96, 32, 16384 - 200, 100, 4, 4, max_blocks=128, max_tokens=16384,
                                        fixed=(31, 32, 63, 64)))
+
+
+def test_qwen_batch1_decode_in_the_benchmark_launch():
+    """The batch-1 Qwen3-4B shape as the benchmark launches it (context 4153, max_tokens 4224): fewer items than
+    warps, so every block of a unit sits on its own warp and the merge gathers the partials of exactly those
+    warps (37 of them, a CTA merge), not of the span between the first and the last."""
+    err = _decode_layer(1, 8, 32, 128, 128, 4096 - 128, 128 + 57, 21, 4, max_blocks=64, max_tokens=4224, samples=3)
+    print("max abs err", err)
+
+
+def test_single_unit_long_context_merges_by_warp():
+    """One (sequence, kv head) over 16421 tokens: 133 partials (129 block items of which 128 hold blocks, and 4
+    tail slots), more than the CTA merge holds in shared memory, so the completing warp merges them alone."""
+    err = _decode_layer(1, 1, 4, 128, 128, 16384 - 128, 128 + 37, 23, 4, max_blocks=129, max_tokens=16512, samples=1)
+    print("max abs err", err)
