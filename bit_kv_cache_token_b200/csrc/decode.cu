@@ -347,8 +347,10 @@ constexpr int kWarpMergeMax = 12;
 // one, whose items sit on separate warps, has the tail spread over up to four.
 constexpr int kTailSlots = kDecodeTailSlots;
 static_assert(kTailSlots * 32 >= kBlockTokens - 1, "the tail slots cover a tail of 127 tokens");
-// Marker of a unit whose merge the completing warp left to its CTA.
-constexpr uint32_t kMergeFlag = 0x80000000u;
+// Most merges a CTA takes over from its warps (its contiguous range touches
+// at most three units that need a CTA merge: one it ends, one it covers
+// whole, one it starts); a warp that finds the list full merges alone.
+constexpr int kCtaMergeCap = 8;
 
 // 2^x for x <= 0 (softmax weights): the hardware approximation, subnormal
 // results flushed to zero (relative error about 2^-22).
@@ -1135,11 +1137,16 @@ decode_kernel(DecodeArgs a, int hb)
     const long long wg = (long long)blockIdx.x * W + warp;
     const long long i_begin = part_begin(wg, total, nw), i_end = part_begin(wg + 1, total, nw);
 
+    // Units whose merge this CTA's warps hand to the CTA (filled by the warp
+    // that completes the unit; read after the CTA's closing barrier).
+    __shared__ int merge_list[kCtaMergeCap];
+    __shared__ int merge_count;
     if (lane == 0) {
         mbar_init(&sm.mbar[0]);
         mbar_init(&sm.mbar[1]);
     }
-    __syncwarp();
+    if (threadIdx.x == 0) merge_count = 0;
+    __syncthreads();
     uint32_t kph = 0u, vph = 0u;
     bool dead = false;  // a staged copy timed out: no more TMA from this warp
 
@@ -1240,57 +1247,26 @@ decode_kernel(DecodeArgs a, int hb)
             __threadfence();
             const UnitSlots us(unit, per_unit, total, nw);
             const int np = us.n + kTailSlots;  // partials to merge
-            if (np <= kWarpMergeMax || np > cta_merge_max<D, GRP>()) {
+            bool alone = np <= kWarpMergeMax || np > cta_merge_max<D, GRP>();
+            if (!alone) {  // hand it to the CTA, whose warps merge it together once they are all done
+                int k = 0;
+                if (lane == 0) {
+                    k = atomicAdd(&merge_count, 1);
+                    if (k < kCtaMergeCap) merge_list[k] = unit;
+                }
+                alone = __shfl_sync(0xffffffffu, k, 0) >= kCtaMergeCap;  // list full: merge alone
+            }
+            if (alone) {
                 warp_merge<D, GRP, MQ>(a, hb, sm, unit, us);
                 if (lane == 0) a.tickets[unit] = 0u;
-            } else if (lane == 0) {
-                atomicExch(a.tickets + unit, kMergeFlag | blockIdx.x);
             }
         }
         i = seg_end;
     }
 
-    // ---- merges left to this CTA: units it touched whose ticket carries its
-    // mark.  Only a unit covered by more than kWarpMergeMax warps (and at most
-    // cta_merge_max) can carry one, and the CTA's contiguous range touches at most three of those (the
-    // first, one covered whole by at least kWarpMergeMax + 1 of its W warps,
-    // the last), so four threads look them up and every thread walks the same list.
-    __shared__ int merge_list[4];
-    __shared__ int merge_count;
+    // ---- the merges this CTA's warps handed over
     __syncthreads();
-    const long long c_begin = part_begin((long long)blockIdx.x * W, total, nw);
-    const long long c_end = part_begin((long long)(blockIdx.x + 1) * W, total, nw);
-    // Candidates: the units of the CTA's range that more than kWarpMergeMax warps
-    // covered; their tickets are read by one thread each, in parallel.
-    __shared__ int merge_flag[4];
-    if (threadIdx.x < 4) {
-        merge_flag[threadIdx.x] = -1;
-        if (c_begin < c_end) {
-            const long long u_first = c_begin / per_unit, u_last = (c_end - 1) / per_unit;
-            long long unit = -1;
-            int k = 0;
-            for (long long u = u_first; u <= u_last; ++u) {  // the threadIdx.x-th candidate
-                const int np = UnitSlots(u, per_unit, total, nw).n + kTailSlots;
-                if (np > kWarpMergeMax && np <= cta_merge_max<D, GRP>()) {
-                    if (k == (int)threadIdx.x) { unit = u; break; }
-                    ++k;
-                }
-            }
-            if (unit >= 0) {
-                __threadfence();
-                if (__ldcg(a.tickets + unit) == (kMergeFlag | blockIdx.x)) merge_flag[threadIdx.x] = (int)unit;
-            }
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int cnt = 0;
-        for (int k = 0; k < 4; ++k)
-            if (merge_flag[k] >= 0) merge_list[cnt++] = merge_flag[k];
-        merge_count = cnt;
-    }
-    __syncthreads();
-    const int nmerge = merge_count;
+    const int nmerge = min(merge_count, kCtaMergeCap);
     for (int j = 0; j < nmerge; ++j) {
         const int unit = merge_list[j];
         cta_merge<D, GRP, MQ>(a, hb, smem_raw, unit, UnitSlots(unit, per_unit, total, nw));
