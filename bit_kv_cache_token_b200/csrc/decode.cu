@@ -248,7 +248,7 @@ __device__ __forceinline__ bool mbar_wait(unsigned long long *bar, uint32_t pari
 // row: channel bits 0-4 pair lanes (shuffles), bits 5 and 6 pair the lane's
 // own values.
 template <int D>
-__device__ void warp_fwht(float *x, int nvec, int hb)
+__device__ __forceinline__ void fwht_rows(float *x, int nvec, int hb)
 {
     constexpr int NV = D / 32;
     const int lane = threadIdx.x & 31;
@@ -288,6 +288,24 @@ __device__ void warp_fwht(float *x, int nvec, int hb)
         for (int i = 0; i < NV; ++i) row[lane + 32 * i] = r[i] * nrm;
     }
     __syncwarp();
+}
+
+// One out-of-line copy of the transform, shared by the query preparation
+// (every segment) and the merges and tails at the end of a launch, which then
+// find it in the instruction cache: about 1 us per launch at GQA 4 (Qwen3-4B
+// shapes, 32K context).  MHA (Phi-3 shapes) ran 1% slower with it and the
+// 8-row instantiation spills around the call, so the others keep inline copies.
+template <int D>
+__device__ __noinline__ void fwht_rows_shared(float *x, int nvec, int hb)
+{
+    fwht_rows<D>(x, nvec, hb);
+}
+
+template <int D, int GRP>
+__device__ __forceinline__ void warp_fwht(float *x, int nvec, int hb)
+{
+    if constexpr (GRP == 4) fwht_rows_shared<D>(x, nvec, hb);
+    else fwht_rows<D>(x, nvec, hb);
 }
 
 
@@ -927,7 +945,7 @@ __device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int u
     for (int hh = 0; hh < GRP; ++hh)
         if (act) *reinterpret_cast<float4 *>(ob + hh * D + c0) = o[hh];
     __syncwarp();
-    warp_fwht<D>(ob, GRP, hb);
+    warp_fwht<D, GRP>(ob, GRP, hb);
 #pragma unroll
     for (int hh = 0; hh < GRP; ++hh) {
         float *row = dst + hh * SR;
@@ -991,7 +1009,7 @@ __device__ void warp_merge(const DecodeArgs &a, int hb, DecWarpSmem<D, GRP> &sm,
         for (int c = 0; c < D / 32; ++c) obuf[hh * D + 32 * c + lane] = acc[c] * linv;
     }
     __syncwarp();
-    warp_fwht<D>(obuf, GRP, hb);
+    warp_fwht<D, GRP>(obuf, GRP, hb);
     if constexpr (MQ) {
 #pragma unroll
         for (int v = 0; v < GRP; ++v) {
@@ -1086,7 +1104,7 @@ __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int 
         obuf[i] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * Li[h];
     }
     __syncthreads();
-    if (warp < GRP) warp_fwht<D>(obuf + warp * D, 1, hb);
+    if (warp < GRP) warp_fwht<D, GRP>(obuf + warp * D, 1, hb);
     __syncthreads();
     if constexpr (MQ) {
         if (tid < GRP * (D / 4)) {  // a float4 of one row per thread
@@ -1188,7 +1206,7 @@ decode_kernel(DecodeArgs a, int hb)
                 for (int j = lane; j < GRP * D; j += 32) (&sm.qbuf[0][0])[j] = In<Tin>::load1(qg + j) * a.scale_log2;
             }
             __syncwarp();
-            warp_fwht<D>(&sm.qbuf[0][0], GRP, hb);
+            warp_fwht<D, GRP>(&sm.qbuf[0][0], GRP, hb);
             const unsigned char *kbase =
                 static_cast<const unsigned char *>(a.k_records) + (size_t)unit * a.max_blocks * R::kBytes;
             const unsigned char *vbase =
