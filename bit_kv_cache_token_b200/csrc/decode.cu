@@ -760,7 +760,7 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
             // MMA chains, interleaved token slice by token slice
 #pragma unroll
             for (int j4 = 0; j4 < kGroup / 8; j4 += 2) {
-                float mine[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                float mine[2][4];
                 CodeWord vw[C][2][2];
                 float acc4[C][2][4];
 #pragma unroll
@@ -794,11 +794,14 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
                 }
                 // the rows of this lane's copy carry the heads of group gg only when cc == copy
 #pragma unroll
-                for (int cc = 0; cc < C; ++cc)
+                for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
-                    for (int jj = 0; jj < 2; ++jj)
+                    for (int i = 0; i < 4; ++i) {
+                        float v = acc4[0][jj][i];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) mine[jj][i] = cc == copy ? acc4[cc][jj][i] : mine[jj][i];
+                        for (int cc = 1; cc < C; ++cc) v = cc == copy ? acc4[cc][jj][i] : v;
+                        mine[jj][i] = v;
+                    }
                 if (gv) {
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
