@@ -116,13 +116,14 @@ __device__ __forceinline__ void split_hilo(float x, float y, uint32_t &hi, uint3
 {
     const __half2 h = __floats2half2_rn(x, y);
     const float2 hf = __half22float2(h);
-    const __half2 l = __floats2half2_rn(x - hf.x, y - hf.y);
+    const float2 d = __ffma2_rn(hf, make_float2(-1.f, -1.f), make_float2(x, y));  // x - hi, exact, both at once
+    const __half2 l = __floats2half2_rn(d.x, d.y);
     hi = *reinterpret_cast<const uint32_t *>(&h);
     lo = *reinterpret_cast<const uint32_t *>(&l);
 }
 
 // hi rows (c0, c1) plus lo rows (c2, c3) of an accumulator
-__device__ __forceinline__ float2 hilo_sum(const float (&c)[4]) { return f2(c[0] + c[2], c[1] + c[3]); }
+__device__ __forceinline__ float2 hilo_sum(const float (&c)[4]) { return __fadd2_rn(f2(c[0], c[1]), f2(c[2], c[3])); }
 
 // Four binary16 values (8 bytes) -> fp32 times `mul`.
 __device__ __forceinline__ float4 h4_to_f4(uint2 w, float mul)
