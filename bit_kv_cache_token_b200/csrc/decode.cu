@@ -710,8 +710,10 @@ __device__ bool run_blocks(DecWarpSmem<D, GRP> &sm, const unsigned char *kbase, 
                 const int T0 = 16 * ks + 2 * tig, T1 = T0 + 8;
                 uint32_t Ab[4] = {0u, 0u, 0u, 0u};
                 if (copy == 0) {
-                    split_hilo(pv[ks][0] * rV[T0], pv[ks][1] * rV[T0 + 1], Ab[0], Ab[1]);
-                    split_hilo(pv[ks][2] * rV[T1], pv[ks][3] * rV[T1 + 1], Ab[2], Ab[3]);
+                    const float2 a0 = __fmul2_rn(f2(pv[ks][0], pv[ks][1]), *reinterpret_cast<const float2 *>(rV + T0));
+                    const float2 a1 = __fmul2_rn(f2(pv[ks][2], pv[ks][3]), *reinterpret_cast<const float2 *>(rV + T1));
+                    split_hilo(a0.x, a0.y, Ab[0], Ab[1]);
+                    split_hilo(a1.x, a1.y, Ab[2], Ab[3]);
                 }
                 uint32_t bb0 = 0u, bb1 = 0u;
                 if (gl < NG) {
