@@ -92,11 +92,13 @@ append_kernel(AppendArgs a)
         status_or(a.status, KVARN_STATUS_CAPACITY);
     }
     __syncthreads();
+    // Arrival: the last of the sequence's 2 * Hkv CTAs advances its length.  It
+    // only has to come after every CTA has read the old length (each read it
+    // before arriving); what the CTAs wrote is read by later launches, which
+    // the kernel boundary orders, so no fence is needed here.
     if (threadIdx.x == 0) {
-        __threadfence();
         const unsigned prev = atomicAdd(a.arrive + s, 1u);
         if (prev == 2u * a.num_kv_heads - 1u) {
-            __threadfence();
             a.arrive[s] = 0u;
             if (!full) a.n_tokens[s] = n + 1;
         }
