@@ -164,8 +164,10 @@ __device__ __forceinline__ void convert_scales(const unsigned char *rec, float *
         o.w = sv[3 * NG + g] * (WITH_R ? rr[3] : 1.f);
         *reinterpret_cast<float4 *>(out_s + g * kBlockTokens + t0) = o;
     }
-    const __half *ch = reinterpret_cast<const __half *>(rec + R::kCOff);
-    for (int d = lane; d < D; d += 32) out_c[d] = __half2float(ch[d]) * cmul;
+    if (4 * lane < D) {  // c of channels 4 lane .. 4 lane + 3 (D <= 128)
+        const uint2 cw = reinterpret_cast<const uint2 *>(rec + R::kCOff)[lane];
+        *reinterpret_cast<float4 *>(out_c + 4 * lane) = h4_to_f4(cw, cmul);
+    }
 }
 
 // The five shifted copies of a code word from which every position is one AND.
@@ -417,8 +419,11 @@ __device__ __forceinline__ void convert_k_scales(const unsigned char *rec, float
         o.w = NG > 3 ? sv[j * NG + 3] * rr[j] : 0.f;
         *reinterpret_cast<float4 *>(srK + 4 * (t0 + j)) = o;
     }
-    const __half *ch = reinterpret_cast<const __half *>(rec + R::kCOff);
-    for (int d = lane; d < D; d += 32) cK[d] = __half2float(ch[d]);
+    // c of channels 4 lane .. 4 lane + 3 (D <= 128): one 8-byte load, one 16-byte store
+    if (4 * lane < D) {
+        const uint2 cw = reinterpret_cast<const uint2 *>(rec + R::kCOff)[lane];
+        *reinterpret_cast<float4 *>(cK + 4 * lane) = h4_to_f4(cw, 1.f);
+    }
 }
 
 // Blocks [b0, b1) of one unit into the running state.  Returns false if a
