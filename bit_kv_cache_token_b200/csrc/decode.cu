@@ -403,21 +403,32 @@ __device__ __forceinline__ void convert_k_scales(const unsigned char *rec, float
     const float4 r4 = h4_to_f4(reinterpret_cast<const uint2 *>(rec + R::kROff)[lane], 1.f);
     *reinterpret_cast<float4 *>(rK + t0) = r4;
     const uint2 *sp = reinterpret_cast<const uint2 *>(rec + R::kSOff) + lane * NG;
-    float sv[4 * NG];
-#pragma unroll
-    for (int i = 0; i < NG; ++i) {
-        const float4 f = h4_to_f4(sp[i], kTwo16);
-        sv[4 * i] = f.x; sv[4 * i + 1] = f.y; sv[4 * i + 2] = f.z; sv[4 * i + 3] = f.w;
-    }
     const float rr[4] = {r4.x, r4.y, r4.z, r4.w};
+    if constexpr (NG == 4) {
+        // token t0 + j's four groups are sp[j]: s times (r 2^16) in packed pairs
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        float4 o;
-        o.x = sv[j * NG] * rr[j];
-        o.y = NG > 1 ? sv[j * NG + 1] * rr[j] : 0.f;
-        o.z = NG > 2 ? sv[j * NG + 2] * rr[j] : 0.f;
-        o.w = NG > 3 ? sv[j * NG + 3] * rr[j] : 0.f;
-        *reinterpret_cast<float4 *>(srK + 4 * (t0 + j)) = o;
+        for (int j = 0; j < 4; ++j) {
+            const float rs = rr[j] * kTwo16;
+            const float2 a = __fmul2_rn(__half22float2(*reinterpret_cast<const __half2 *>(&sp[j].x)), f2(rs, rs));
+            const float2 b = __fmul2_rn(__half22float2(*reinterpret_cast<const __half2 *>(&sp[j].y)), f2(rs, rs));
+            *reinterpret_cast<float4 *>(srK + 4 * (t0 + j)) = make_float4(a.x, a.y, b.x, b.y);
+        }
+    } else {
+        float sv[4 * NG];
+#pragma unroll
+        for (int i = 0; i < NG; ++i) {
+            const float4 f = h4_to_f4(sp[i], kTwo16);
+            sv[4 * i] = f.x; sv[4 * i + 1] = f.y; sv[4 * i + 2] = f.z; sv[4 * i + 3] = f.w;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float4 o;
+            o.x = sv[j * NG] * rr[j];
+            o.y = NG > 1 ? sv[j * NG + 1] * rr[j] : 0.f;
+            o.z = NG > 2 ? sv[j * NG + 2] * rr[j] : 0.f;
+            o.w = NG > 3 ? sv[j * NG + 3] * rr[j] : 0.f;
+            *reinterpret_cast<float4 *>(srK + 4 * (t0 + j)) = o;
+        }
     }
     // c of channels 4 lane .. 4 lane + 3 (D <= 128): one 8-byte load, one 16-byte store
     if (4 * lane < D) {
