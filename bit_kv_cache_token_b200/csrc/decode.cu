@@ -1007,28 +1007,62 @@ __device__ void warp_merge(const DecodeArgs &a, int hb, DecWarpSmem<D, GRP> &sm,
     const int lane = threadIdx.x & 31;
     float *obuf = reinterpret_cast<float *>(sm.rec[0]);  // [GRP][D]
     const int P = us.n + kTailSlots;
+    // lanes over partials: the largest m of every head
+    float M[GRP];
+#pragma unroll
+    for (int hh = 0; hh < GRP; ++hh) M[hh] = -INFINITY;
+    for (int p = lane; p < P; p += 32) {
+        const float *row = unit_partial<D, GRP>(a, unit, us, p);
+#pragma unroll
+        for (int hh = 0; hh < GRP; ++hh) M[hh] = fmaxf(M[hh], __ldcg(row + hh * SR));
+    }
+#pragma unroll
+    for (int hh = 0; hh < GRP; ++hh)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M[hh] = fmaxf(M[hh], __shfl_xor_sync(0xffffffffu, M[hh], o));
+    // 32 partials at a time: lane j fetches partial p0 + j's row address, weights and l, which the
+    // warp then takes in order by shuffles; the rows' loads do not wait on one another
+    float L[GRP], acc[GRP][D / 32];
+#pragma unroll
     for (int hh = 0; hh < GRP; ++hh) {
-        // lanes over partials: the maximum, then weights and the normaliser
-        float M = -INFINITY;
-        for (int p = lane; p < P; p += 32) M = fmaxf(M, __ldcg(unit_partial<D, GRP>(a, unit, us, p) + hh * SR));
+        L[hh] = 0.f;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        float L = 0.f;
-        float acc[D / 32];
+        for (int c = 0; c < D / 32; ++c) acc[hh][c] = 0.f;
+    }
+    for (int p0 = 0; p0 < P; p0 += 32) {
+        const int p = p0 + lane;
+        const float *row = unit_partial<D, GRP>(a, unit, us, p < P ? p : p0);
+        float w[GRP], lv[GRP];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) acc[c] = 0.f;
-        for (int p = 0; p < P; ++p) {
-            const float *row = unit_partial<D, GRP>(a, unit, us, p) + hh * SR;
-            const float m = __ldcg(row);
-            const float wgt = (M > -INFINITY && m > -INFINITY) ? exp2f(m - M) : 0.f;
-            if (wgt == 0.f) continue;
-            L = fmaf(__ldcg(row + 1), wgt, L);
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) acc[c] = fmaf(__ldcg(row + 4 + 32 * c + lane), wgt, acc[c]);
+        for (int hh = 0; hh < GRP; ++hh) {
+            const float m = p < P ? __ldcg(row + hh * SR) : -INFINITY;
+            w[hh] = (M[hh] > -INFINITY && m > -INFINITY) ? exp2f(m - M[hh]) : 0.f;
+            lv[hh] = p < P ? __ldcg(row + hh * SR + 1) : 0.f;
         }
-        const float linv = L > 0.f ? 1.f / L : 0.f;
+        const unsigned long long ra = reinterpret_cast<unsigned long long>(row);
+        const int nj = min(32, P - p0);
+#pragma unroll 4
+        for (int j = 0; j < nj; ++j) {
+            const float *rj = reinterpret_cast<const float *>(__shfl_sync(0xffffffffu, ra, j));
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) obuf[hh * D + 32 * c + lane] = acc[c] * linv;
+            for (int hh = 0; hh < GRP; ++hh) {
+                const float wj = __shfl_sync(0xffffffffu, w[hh], j);
+                const float lj = __shfl_sync(0xffffffffu, lv[hh], j);
+                // a partial of weight 0 (empty, or far below the maximum) is left out
+                L[hh] = wj == 0.f ? L[hh] : fmaf(lj, wj, L[hh]);
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    const float x = __ldcg(rj + hh * SR + 4 + 32 * c + lane);
+                    acc[hh][c] = wj == 0.f ? acc[hh][c] : fmaf(x, wj, acc[hh][c]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int hh = 0; hh < GRP; ++hh) {
+        const float linv = L[hh] > 0.f ? 1.f / L[hh] : 0.f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) obuf[hh * D + 32 * c + lane] = acc[hh][c] * linv;
     }
     __syncwarp();
     warp_fwht<D, GRP>(obuf, GRP, hb);
@@ -1074,21 +1108,17 @@ __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int 
     float *Mh = Li + GP;                             // [GRP]
     float *wts = Mh + GP;                            // [P][GRP] weights exp2(m - M)
 
-    // ---- one round of copies: the block partials, then the tail partials
-    {
-        const int nb16 = us.n * SLOT / 4, n16 = P * SLOT / 4;  // SLOT is a multiple of 4 floats
-        const bool contiguous = us.total >= us.nw;  // block partials in slots wf + unit .. wf + unit + n - 1
-        for (int i = tid; i < n16; i += NT) {
-            const float *g;
-            if (i >= nb16) g = a.tail_partials + (size_t)unit * kTailSlots * SLOT + 4 * (size_t)(i - nb16);
-            else if (contiguous) g = a.partials + (size_t)(us.wf + unit) * SLOT + 4 * (size_t)i;
-            else g = a.partials + (size_t)(us.warp(i / (SLOT / 4)) + unit) * SLOT + 4 * (i % (SLOT / 4));
-            const uint32_t d = smem_u32(parts + 4 * (size_t)i);
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(g) : "memory");
-        }
-        asm volatile("cp.async.commit_group;\n" ::: "memory");
-        asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+    // ---- one round of copies: the block partials, then the tail partials (a warp per
+    // partial, whose slot address is worked out once; lanes over its 16-byte pieces)
+    static_assert(SLOT % 4 == 0, "a partial is a whole number of 16-byte pieces");
+    for (int p = warp; p < P; p += W) {
+        const float *g = unit_partial<D, GRP>(a, unit, us, p);
+        const uint32_t d = smem_u32(parts + (size_t)p * SLOT);
+        for (int c = lane; c < SLOT / 4; c += 32)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d + 16 * c), "l"(g + 4 * c) : "memory");
     }
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
     __syncthreads();
     // ---- per head: the largest m, the weights and the normaliser (warp h for head h)
     for (int h = warp; h < GRP; h += W) {
@@ -1112,18 +1142,32 @@ __device__ void cta_merge(const DecodeArgs &a, int hb, unsigned char *smem, int 
         }
     }
     __syncthreads();
-    // ---- weighted sum of the partials (an empty partial has weight 0 and zero rows)
-    for (int i = tid; i < GRP * D; i += NT) {
-        const int h = i / D, c = i % D;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains
+    // ---- weighted sum of the partials (an empty partial has weight 0 and zero rows), four
+    // channels a thread, two chains over the partials
+    for (int i = tid; i < GRP * (D / 4); i += NT) {
+        const int h = i / (D / 4), c = 4 * (i % (D / 4));
+        const float *src = parts + h * SR + 4 + c;
+        float2 a01 = f2(0.f, 0.f), a23 = f2(0.f, 0.f), b01 = f2(0.f, 0.f), b23 = f2(0.f, 0.f);
         int p = 0;
-        for (; p + 3 < P; p += 4) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                acc[e] = fmaf(wts[(p + e) * GRP + h], parts[(size_t)(p + e) * SLOT + h * SR + 4 + c], acc[e]);
+        for (; p + 1 < P; p += 2) {
+            const float w0 = wts[p * GRP + h], w1 = wts[(p + 1) * GRP + h];
+            const float4 x0 = *reinterpret_cast<const float4 *>(src + (size_t)p * SLOT);
+            const float4 x1 = *reinterpret_cast<const float4 *>(src + (size_t)(p + 1) * SLOT);
+            a01 = __ffma2_rn(f2(x0.x, x0.y), f2(w0, w0), a01);
+            a23 = __ffma2_rn(f2(x0.z, x0.w), f2(w0, w0), a23);
+            b01 = __ffma2_rn(f2(x1.x, x1.y), f2(w1, w1), b01);
+            b23 = __ffma2_rn(f2(x1.z, x1.w), f2(w1, w1), b23);
         }
-        for (; p < P; ++p) acc[0] = fmaf(wts[p * GRP + h], parts[(size_t)p * SLOT + h * SR + 4 + c], acc[0]);
-        obuf[i] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * Li[h];
+        if (p < P) {
+            const float w0 = wts[p * GRP + h];
+            const float4 x0 = *reinterpret_cast<const float4 *>(src + (size_t)p * SLOT);
+            a01 = __ffma2_rn(f2(x0.x, x0.y), f2(w0, w0), a01);
+            a23 = __ffma2_rn(f2(x0.z, x0.w), f2(w0, w0), a23);
+        }
+        const float li = Li[h];
+        const float2 o01 = __fmul2_rn(__fadd2_rn(a01, b01), f2(li, li));
+        const float2 o23 = __fmul2_rn(__fadd2_rn(a23, b23), f2(li, li));
+        *reinterpret_cast<float4 *>(obuf + h * D + c) = make_float4(o01.x, o01.y, o23.x, o23.y);
     }
     __syncthreads();
     if (warp < GRP) warp_fwht<D, GRP>(obuf + warp * D, 1, hb);
