@@ -226,6 +226,12 @@ __device__ __forceinline__ bool mbar_try(unsigned long long *bar, uint32_t parit
     return done != 0u;
 }
 
+// A hint that the 128-byte line holding p be brought into L2.
+__device__ __forceinline__ void prefetch_l2(const void *p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ unsigned long long global_ns()
 {
     unsigned long long t;
@@ -862,6 +868,15 @@ __device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int u
     static_assert(sizeof(float) * kBlockTokens * GRP <= sizeof(sm.rec), "tail scratch");
     const int nt = t1 - t0;
     if (nt > 0) {
+        // the range's K and V rows are prefetched into L2 while the query is staged
+        const Tin *kt = static_cast<const Tin *>(a.k_tail) + (size_t)unit * kBlockTokens * D;
+        const Tin *vt0 = static_cast<const Tin *>(a.v_tail) + (size_t)unit * kBlockTokens * D;
+        constexpr int kLines = (D * (int)sizeof(Tin) + 127) / 128;  // 128-byte lines per row
+        for (int i = lane; i < nt * kLines; i += 32) {
+            const size_t off = (size_t)(t0 + i / kLines) * D * sizeof(Tin) + 128 * (i % kLines);
+            prefetch_l2(reinterpret_cast<const unsigned char *>(kt) + off);
+            prefetch_l2(reinterpret_cast<const unsigned char *>(vt0) + off);
+        }
         if constexpr (MQ) {
 #pragma unroll
             for (int v = 0; v < GRP; ++v) {
@@ -874,7 +889,6 @@ __device__ void tail_partial(const DecodeArgs &a, DecWarpSmem<D, GRP> &sm, int u
         }
         __syncwarp();
         // scores: lanes over tokens, a row's loads issued together
-        const Tin *kt = static_cast<const Tin *>(a.k_tail) + (size_t)unit * kBlockTokens * D;
         for (int u0 = 0; u0 < nt; u0 += 32) {
             const int u = u0 + lane, t = t0 + u;
             if (u < nt) {
