@@ -49,7 +49,7 @@ QB_WORKLOAD = "Llama-3-8B-shaped bulk prefill quantise: 32 batch x 32 layers x 8
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one decode launch at context 32705 for this
 # batch, from one ncu capture of `bench.py --profile decode` with the current decode kernel; None whenever
 # the decode kernel has changed since the last capture.
-DECODE_TRAFFIC_BYTES = 220198656 + 4261888
+DECODE_TRAFFIC_BYTES = 220170496 + 4353280
 # The same for one bulk-quantisation launch of `bench.py --profile quantize` (16 of the 1024 sequences); the
 # traffic grows with the sequences, so the full workload's is 64 times this.
 QUANT_TRAFFIC_BYTES_16SEQ = 537332992 + 97235968

@@ -1223,6 +1223,7 @@ decode_kernel(DecodeArgs a, int hb)
     constexpr int NTN = (GRP + 3) / 4;
     constexpr int SR = slot_row<D>();
     extern __shared__ __align__(128) unsigned char smem_raw[];
+    grid_dep_wait();  // the previous kernel in the stream (an append, say) has completed
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     DecWarpSmem<D, GRP> &sm = reinterpret_cast<DecWarpSmem<D, GRP> *>(smem_raw)[warp];
     const int gl = lane >> 2, tig = lane & 3;
@@ -1380,8 +1381,8 @@ static cudaError_t launch_dec_mq(const DecodeArgs &a, int hb, int ctas, cudaStre
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, GRP, Tin, MQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    decode_kernel<D, GRP, Tin, MQ><<<ctas, W * 32, smem, st>>>(a, hb);
-    return cudaGetLastError();
+    e = launch_overlapped(decode_kernel<D, GRP, Tin, MQ>, dim3(ctas), dim3(W * 32), smem, st, a, hb);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // One query per sequence (the common case) runs the kernel without the

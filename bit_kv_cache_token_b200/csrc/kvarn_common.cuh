@@ -135,4 +135,33 @@ __device__ __forceinline__ void status_or(int32_t *status, int bits)
     if (status) atomicOr(reinterpret_cast<int *>(status), bits);
 }
 
+// Programmatic dependent launch.  A kernel launched by launch_overlapped has
+// its launch prepared while the kernel before it in the stream is still
+// running; grid_dep_wait blocks until that kernel has completed and its
+// writes are visible, so it comes before the kernel's first access to global
+// memory (in a kernel launched the ordinary way it returns at once).  No
+// kernel here releases its dependents early (griddepcontrol.launch_dependents):
+// with an early release the next kernel's blocks took the first SMs that the
+// running kernel's blocks left, several to an SM, and the Qwen3-4B-shaped
+// batch-8 step ran 0.7-4% slower; without it the step runs 0.6% faster than
+// with ordinary launches.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                     Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 }  // namespace kvarn

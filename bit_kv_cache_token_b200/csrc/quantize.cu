@@ -65,6 +65,7 @@ template <int D, int HB, typename Tin>
 __global__ void __launch_bounds__(D, 2)
 append_kernel(AppendArgs a)
 {
+    grid_dep_wait();  // the previous kernel in the stream (a decode, say) has completed
     QuantSmem<D> &sm = quant_smem<D>();
     __shared__ int s_n;
     const int sh = blockIdx.x;  // s * Hkv + h
@@ -132,8 +133,8 @@ static cudaError_t launch_append(const AppendArgs &a, int S, int Hkv, cudaStream
     if (e != cudaSuccess) return e;
     // the largest shared-memory carveout, so that three CTAs fit on an SM
     cudaFuncSetAttribute(append_kernel<D, HB, Tin>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    append_kernel<D, HB, Tin><<<grid, D, kSmem, st>>>(a);
-    return cudaGetLastError();
+    const cudaError_t el = launch_overlapped(append_kernel<D, HB, Tin>, grid, dim3(D), (size_t)kSmem, st, a);
+    return el != cudaSuccess ? el : cudaGetLastError();
 }
 
 // ---- dispatch over (D, Hadamard block, dtype) ---------------------------
