@@ -80,7 +80,8 @@ __host__ __device__ constexpr int dec_sets()
     return (D / kGroup + 8 / GRP - 1) / (8 / GRP);
 }
 
-// Warps per CTA: up to 12, as many as fit in 227 KB of shared memory.
+// Warps per CTA: up to 12 (16 for one row per kv head, 8 for eight rows), as
+// many as fit in 227 KB of shared memory.
 template <int D, int GRP>
 __host__ __device__ constexpr int dec_warps()
 {
@@ -88,9 +89,13 @@ __host__ __device__ constexpr int dec_warps()
     // SM all leave 168 registers a thread.  The 8-row instantiation needs
     // more than that (it spills over 200 bytes at 168), so it runs 8 warps
     // with up to 255 registers and no spills: 156 against 170 us for two
-    // query tokens at 32705 cached tokens (Qwen3-4B shapes, batch 8).
+    // query tokens at 32705 cached tokens (Qwen3-4B shapes, batch 8).  One
+    // row per kv head (MHA) needs fewer: where 16 warps fit in shared memory
+    // (head_dim 64 and 96) it runs 16 with 128 registers, a few words spilled
+    // at head_dim 96: 257 against 279 us per Phi-3-mini-shaped layer (batch
+    // 16, 32 heads, 16384 tokens).
     constexpr int fit = (227 * 1024) / (int)sizeof(DecWarpSmem<D, GRP>);
-    constexpr int cap = GRP == 8 ? 8 : 12;
+    constexpr int cap = GRP == 8 ? 8 : (GRP == 1 && fit >= 16) ? 16 : 12;
     return fit < cap ? fit : cap;
 }
 
